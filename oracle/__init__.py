@@ -1,0 +1,213 @@
+"""CPU oracle for key-priority mixed-precision KV-cache quantization.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference leg of ``bench.py`` may import this package.  The
+product path (``kv_cache_mixed_kvq_b200``) never imports it and shares no code
+with it: the C source next to this file restates the quantizer, the cache
+format and attention from their definitions.
+
+Functions follow "Quantize What Counts: More for Keys, Less for Values"
+(summary page): keys and values quantized with separate bit widths
+("Key contributions", K4V2 etc.), group-wise ("Results", "Group-size
+sensitivity"), and attention over the dequantised cache ("Problem
+statement": the cache is what inference reads).  See ``kvq_oracle.c`` for the
+step-by-step definitions.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvq_oracle.c")
+_LIB = os.path.join(_HERE, "libkvq_oracle.so")
+
+DTYPE_CODE = {"f32": 0, "bf16": 1, "f16": 2}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call([
+            "gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+            "-fPIC", "-shared", _SRC, "-o", tmp, "-lm",
+        ])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load(path: str | None = None):
+    lib = ctypes.CDLL(path or build())
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    lib.ora_f32_to_f16.argtypes = [ctypes.c_float]
+    lib.ora_f32_to_f16.restype = ctypes.c_uint16
+    lib.ora_f16_to_f32.argtypes = [ctypes.c_uint16]
+    lib.ora_f16_to_f32.restype = ctypes.c_float
+    lib.ora_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    lib.ora_bf16_to_f32.restype = ctypes.c_float
+    lib.ora_quantize_group.argtypes = [P, I, I, P, P, P, P, P]
+    lib.ora_quantize_group.restype = None
+    lib.ora_k_code_place.argtypes = [I, I, I, P, P]
+    lib.ora_v_code_place.argtypes = [I, I, I, I, P, P]
+    lib.ora_quantize_append.argtypes = [I] * 7 + [P] * 6 + [I, P, I]
+    lib.ora_quantize_append.restype = I
+    lib.ora_read_codes.argtypes = [I, I, I, I, I, P, P, I, I, I, I, P]
+    lib.ora_dequant_row.argtypes = [I, I, I, I, I, I, P, P, P, P, I, I, I, I, P]
+    lib.ora_decode_attention.argtypes = [I] * 7 + [P] * 4 + [P, I, I, P, I, ctypes.c_float, P]
+    lib.ora_decode_attention.restype = I
+    lib.ora_attention_dense.argtypes = [I, I, I, I, P, P, I, P, I, I, P, ctypes.c_float, P]
+    lib.ora_attention_dense.restype = I
+    return lib
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_of(a: np.ndarray, dtype: str | None) -> str:
+    if dtype is not None:
+        return dtype
+    if a.dtype == np.float32:
+        return "f32"
+    raise ValueError("16-bit inputs are passed as uint16 bit patterns with dtype='bf16' or 'f16'")
+
+
+# ------------------------------------------------------------------ numbers
+def f32_to_f16_bits(x: float) -> int:
+    return int(lib().ora_f32_to_f16(float(x)))
+
+
+def f16_bits_to_f32(h: int) -> float:
+    return float(lib().ora_f16_to_f32(int(h)))
+
+
+def bf16_bits_to_f32(h: int) -> float:
+    return float(lib().ora_bf16_to_f32(int(h)))
+
+
+# ---------------------------------------------------------------- quantizer
+def quantize_group(x, bits: int):
+    """Codes, binary32 scale and min, binary16 scale/zero bits of one group."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    codes = np.zeros(x.size, np.uint8)
+    s32 = np.zeros(1, np.float32)
+    m32 = np.zeros(1, np.float32)
+    s16 = np.zeros(1, np.uint16)
+    z16 = np.zeros(1, np.uint16)
+    lib().ora_quantize_group(_ptr(x), x.size, bits, _ptr(codes), _ptr(s32), _ptr(m32),
+                             _ptr(s16), _ptr(z16))
+    return codes, float(s32[0]), float(m32[0]), int(s16[0]), int(z16[0])
+
+
+def k_code_place(D: int, bits: int, d: int):
+    off = ctypes.c_int()
+    sh = ctypes.c_int()
+    lib().ora_k_code_place(D, bits, d, ctypes.byref(off), ctypes.byref(sh))
+    return off.value, sh.value
+
+
+def v_code_place(D: int, bits: int, k: int, d: int):
+    off = ctypes.c_int()
+    sh = ctypes.c_int()
+    lib().ora_v_code_place(D, bits, k, d, ctypes.byref(off), ctypes.byref(sh))
+    return off.value, sh.value
+
+
+# ------------------------------------------------------------------- cache
+class HostCache:
+    """Host copies of the four cache arrays in the library's format."""
+
+    def __init__(self, B, Hkv, D, capacity, bits_k, bits_v, group):
+        self.B, self.Hkv, self.D, self.cap = B, Hkv, D, capacity
+        self.bits_k, self.bits_v, self.group = bits_k, bits_v, group
+        slots = B * Hkv
+        self.k_codes = np.zeros(slots * capacity * D * bits_k // 8, np.uint8)
+        self.v_codes = np.zeros(slots * capacity * D * bits_v // 8, np.uint8)
+        ng = D // group
+        self.k_params = np.zeros(slots * capacity * ng * 2, np.uint16)
+        self.v_params = np.zeros(slots * capacity * ng * 2, np.uint16)
+
+    def _shape(self):
+        return (self.B, self.Hkv, self.D, self.cap, self.bits_k, self.bits_v, self.group)
+
+    def quantize_append(self, k: np.ndarray, v: np.ndarray, pos, dtype: str | None = None) -> int:
+        """k, v: [B][Hkv][n_new][D] float32 or uint16 bit patterns."""
+        k = np.ascontiguousarray(k)
+        v = np.ascontiguousarray(v)
+        n_new = k.shape[2]
+        assert k.shape == (self.B, self.Hkv, n_new, self.D) and v.shape == k.shape
+        pos = np.ascontiguousarray(pos, dtype=np.int32)
+        dt = DTYPE_CODE[_dtype_of(k, dtype)]
+        r = lib().ora_quantize_append(*self._shape(), _ptr(self.k_codes), _ptr(self.v_codes),
+                                      _ptr(self.k_params), _ptr(self.v_params),
+                                      _ptr(k), _ptr(v), dt, _ptr(pos), n_new)
+        if r < 0:
+            raise ValueError("invalid cache shape")
+        return r
+
+    def read_codes(self, which: int, b: int, h: int, p: int) -> np.ndarray:
+        out = np.zeros(self.D, np.uint8)
+        lib().ora_read_codes(self.Hkv, self.D, self.cap, self.bits_k, self.bits_v,
+                             _ptr(self.k_codes), _ptr(self.v_codes), which, b, h, p, _ptr(out))
+        return out
+
+    def dequant_row(self, which: int, b: int, h: int, p: int) -> np.ndarray:
+        out = np.zeros(self.D, np.float32)
+        lib().ora_dequant_row(self.Hkv, self.D, self.cap, self.bits_k, self.bits_v, self.group,
+                              _ptr(self.k_codes), _ptr(self.v_codes), _ptr(self.k_params),
+                              _ptr(self.v_params), which, b, h, p, _ptr(out))
+        return out
+
+    def dequant_slot(self, which: int, b: int, h: int, n: int) -> np.ndarray:
+        return np.stack([self.dequant_row(which, b, h, p) for p in range(n)]) if n else \
+            np.zeros((0, self.D), np.float32)
+
+    def decode_attention(self, q: np.ndarray, Hq: int, seq_lens, sm_scale: float = 0.0,
+                         q_dtype: str | None = None, max_len: int | None = None):
+        """Returns (out float64 [B][Hq][D], flags)."""
+        q = np.ascontiguousarray(q)
+        assert q.shape == (self.B, Hq, self.D)
+        lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        out = np.zeros((self.B, Hq, self.D), np.float64)
+        r = lib().ora_decode_attention(*self._shape(), _ptr(self.k_codes), _ptr(self.v_codes),
+                                       _ptr(self.k_params), _ptr(self.v_params), _ptr(q),
+                                       DTYPE_CODE[_dtype_of(q, q_dtype)], Hq, _ptr(lens),
+                                       self.cap if max_len is None else max_len,
+                                       float(sm_scale), _ptr(out))
+        if r < 0:
+            raise ValueError("invalid shape")
+        return out, r
+
+
+def attention_dense(k: np.ndarray, v: np.ndarray, q: np.ndarray, seq_lens, sm_scale: float = 0.0,
+                    kv_dtype: str | None = None, q_dtype: str | None = None) -> np.ndarray:
+    """Unquantised attention: k, v [B][Hkv][T][D], q [B][Hq][D] -> float64."""
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    q = np.ascontiguousarray(q)
+    B, Hkv, T, D = k.shape
+    Hq = q.shape[1]
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    out = np.zeros((B, Hq, D), np.float64)
+    r = lib().ora_attention_dense(B, Hkv, D, T, _ptr(k), _ptr(v), DTYPE_CODE[_dtype_of(k, kv_dtype)],
+                                  _ptr(q), DTYPE_CODE[_dtype_of(q, q_dtype)], Hq, _ptr(lens),
+                                  float(sm_scale), _ptr(out))
+    if r < 0:
+        raise ValueError("invalid shape")
+    return out
