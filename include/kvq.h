@@ -22,8 +22,9 @@
  *
  * Quantizer (per row r = (batch, kv_head, token), per group of G elements,
  * every step in IEEE binary32, round-to-nearest-even, no fused multiply-add):
- *   1. mn = min x_i, mx = max x_i over the group; then mn = mn + 0.0f
- *      (so that a -0 minimum is stored as +0).
+ *   1. mn = min x_i, mx = max x_i over the group; then mn = mn + 0.0f and
+ *      mx = mx + 0.0f (a zero extreme is +0 whatever the order of reduction,
+ *      so the stored binary16 patterns are unique).
  *   2. range = mx - mn;  scale = range / (2^b - 1);  inv = 1 / scale.
  *   3. If scale == 0, or scale or inv is not finite, every code is 0
  *      (degenerate group).  Otherwise

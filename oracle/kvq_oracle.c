@@ -16,8 +16,8 @@
  *     the summary page "Quantize What Counts: More for Keys, Less for Values"
  *     leaves open ("Problem statement": BF16 cache stored at INT4 or fewer
  *     bits; "Results", "Group-size sensitivity": one quantizer per group of
- *     head_dim elements).  Steps in binary32, in this order: min/max,
- *     range/(2^b-1), reciprocal, (x-min)*reciprocal, round half to even,
+ *     head_dim elements).  Steps in binary32, in this order: min/max
+ *     (signed zeros made +0), range/(2^b-1), reciprocal, (x-min)*reciprocal, round half to even,
  *     clamp; stored scale and min rounded to binary16.
  *   - ora_k_code_place / ora_v_code_place: where a code lives in the packed
  *     cache (the library's documented format; see the header of the library
@@ -109,6 +109,7 @@ void ora_quantize_group(const float* x, int n, int bits, uint8_t* codes,
     if (x[i] > mx) mx = x[i];
   }
   mn = mn + 0.0f; /* a -0 minimum becomes +0 */
+  mx = mx + 0.0f; /* and so does a -0 maximum */
   float levels = (float)((1 << bits) - 1);
   float range = mx - mn;
   float scale = range / levels;

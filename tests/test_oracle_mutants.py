@@ -24,6 +24,7 @@ MUTANTS = {
     "levels_off_by_one": ("float levels = (float)((1 << bits) - 1);",
                           "float levels = (float)(1 << bits);"),
     "no_negative_zero_fix": ("mn = mn + 0.0f; /* a -0 minimum becomes +0 */", ""),
+    "no_negative_zero_fix_max": ("mx = mx + 0.0f; /* and so does a -0 maximum */", ""),
     "k_slice_index": ("int slice = (d % 8) / 2;", "int slice = d % 4;"),
     "v_half_swapped": ("int bit = 16 * (k % 2) + b * ((d / 8) % E);\n  int n",
                        "int bit = 16 * (1 - k % 2) + b * ((d / 8) % E);\n  int n"),
@@ -43,6 +44,7 @@ PINS = [
     lambda o: qz.test_exact_grid(o, 2),
     lambda o: qz.test_ties_round_half_even(o),
     lambda o: qz.test_negative_zero_minimum_is_canonical(o),
+    lambda o: qz.test_signed_zero_extremes_give_positive_zero_params(o),
     lambda o: qz.test_codes_are_nearest_levels_exact_rationals(o, 4),
     lambda o: qz.test_cache_dequant_within_error_bound(o, 0, 4),
     lambda o: lay.test_k_row_fields_tile_the_row(o, 128, 4),

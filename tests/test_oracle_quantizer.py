@@ -57,6 +57,16 @@ def test_negative_zero_minimum_is_canonical(ora):
     assert codes.tolist() == [0, 1, 2, 3]
 
 
+def test_signed_zero_extremes_give_positive_zero_params(ora):
+    # all-zero group with mixed signs: range +0, scale +0, zero +0
+    for x in ([-0.0, 0.0, -0.0], [0.0, -0.0], [-0.0, -0.0]):
+        codes, s32, m32, s16, z16 = ora.quantize_group(np.array(x, np.float32), 4)
+        assert (s16, z16) == (0x0000, 0x0000) and not codes.any()
+    # negative group whose maximum is -0: range = 0 - mn
+    codes, s32, m32, s16, z16 = ora.quantize_group(np.array([-3.0, -0.0], np.float32), 2)
+    assert s32 == 1.0 and codes.tolist() == [0, 3]
+
+
 def test_subnormal_range_degenerates(ora):
     # range 2^-140: scale is subnormal and 1/scale overflows -> all codes 0
     x = np.array([0.0, 2.0 ** -140], np.float32)
