@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Benchmark of the mixed-precision KV-cache hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+quantize-append (group-wise min-max, keys at b_k and values at b_v bits,
+bit-packed) followed by split-K decode attention over the packed cache and
+the log-sum-exp combine.  Default workload: the Llama-3-8B-shaped decode
+layer (batch 8, 32 query / 8 KV heads, head_dim 128, 4096 tokens per
+sequence, bf16, K4V2, group 64), quantizing the full cache then one decode
+step.  Other workloads (`--workload`) append their new tokens and decode.
+
+Timing: inputs and caches rotate over enough sets that no step finds its data
+in L2; each step is replayed from a CUDA graph; the timed region is bracketed
+by a barrier and a device synchronize, timed with CUDA events on the launch
+stream, max over ranks.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_mixed_kvq_b200 import workloads  # noqa: E402
+
+METRIC = "quantized-KV decode attention HBM GB/s (% of B200 peak) and KV-tokens/s, K4V2"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------- workload
+def step_shape(w: workloads.Workload, bits):
+    """Sizes of one step: new tokens written per sequence and lengths read."""
+    lens = workloads.seq_lens(w).tolist()
+    if w.name == "llama3_8b":
+        n_new, pos = w.context, [0] * w.batch          # quantize the full cache
+        read = lens
+    else:
+        n_new = max(w.append, 0)
+        pos = [n - n_new for n in lens] if n_new else lens
+        read = lens
+    return n_new, pos, read
+
+
+def algorithmic_bytes(w: workloads.Workload, bits, n_new, read_lens):
+    """HBM bytes the step must move, by kernel (what the method reads/writes)."""
+    bk, bv = bits
+    D, G = w.head_dim, w.group
+    el = 4 if w.dtype == "f32" else 2
+    per_tok_cache = D * (bk + bv) // 8 + 2 * (D // G) * 4
+    rows = w.batch * w.kv_heads * n_new
+    quant = rows * (2 * D * el + per_tok_cache) + 4 * w.batch
+    tokens = sum(read_lens)
+    decode = tokens * w.kv_heads * per_tok_cache + 2 * w.batch * w.q_heads * D * el + 4 * w.batch
+    return {"quantize": quant, "decode": decode, "tokens": tokens, "per_token_head": per_tok_cache}
+
+
+def sha_of(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {
+    "quantize": ["kv_cache_mixed_kvq_b200/csrc/quantize.cu", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
+    "decode": ["kv_cache_mixed_kvq_b200/csrc/decode.cuh", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
+}
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it still
+    matches the kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            data = json.load(f)
+    except (OSError, ValueError):
+        return None
+    rec = data.get(f"{kernel}/{workload}")
+    if not rec or rec.get("source_sha") != sha_of(KERNEL_SOURCES[kernel]):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        rows = [[x.strip() for x in r] for r in rows if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# -------------------------------------------------------------- our arm
+class Arm:
+    """Device buffers for R rotating sets of inputs + caches, and the step."""
+
+    def __init__(self, w, bits, rotate: int, device):
+        import kv_cache_mixed_kvq_b200 as kvq
+        self.kvq = kvq
+        self.w, self.bits = w, bits
+        self.n_new, self.pos, self.read = step_shape(w, bits)
+        self.cap = w.capacity()
+        self.lens = torch.tensor(self.read, dtype=torch.int32, device=device)
+        self.max_len = max(self.read)
+        self.pos_t = torch.tensor(self.pos, dtype=torch.int32, device=device)
+        self.sets = []
+        for r in range(rotate):
+            cache = kvq.KVCache.allocate(w.batch, w.kv_heads, w.head_dim, self.cap, bits[0],
+                                         bits[1], w.group, device=device)
+            if w.name != "llama3_8b":
+                # pre-fill the context (untimed); the step then appends n_new tokens
+                for b in range(w.batch):
+                    kb, vb = workloads.make_kv(w, self.read[b], seed=100 + r * 1000 + b,
+                                               device=device, batch=1)
+                    kvq.kvq_quantize_append(_slot_view(cache, b), kb, vb,
+                                            torch.zeros(1, dtype=torch.int32, device=device))
+            k, v = workloads.make_kv(w, max(self.n_new, 1), seed=r, device=device)
+            q = workloads.make_q(w, seed=r, device=device)
+            out = torch.empty_like(q)
+            self.sets.append(dict(cache=cache, k=k, v=v, q=q, out=out))
+        ws = kvq.kvq_decode_workspace_bytes(self.sets[0]["cache"], w.q_heads, self.max_len)
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+        self.split_tokens = kvq.kvq_decode_split_tokens(self.sets[0]["cache"], w.q_heads,
+                                                        self.max_len)
+
+    def quantize(self, r):
+        s = self.sets[r]
+        if self.n_new:
+            self.kvq.kvq_quantize_append(s["cache"], s["k"], s["v"], self.pos_t)
+
+    def decode(self, r):
+        s = self.sets[r]
+        self.kvq.kvq_decode_attention(s["cache"], s["q"], self.lens, self.max_len, out=s["out"],
+                                      workspace=self.ws)
+
+    def step(self, r):
+        self.quantize(r)
+        self.decode(r)
+
+    launches_per_step = property(lambda self: (1 if self.n_new else 0) + 2)
+
+
+def _slot_view(cache, b):
+    """A KVCache over batch row b only (views into the same buffers)."""
+    per = [t.numel() // cache.batch for t in (cache.k_codes, cache.v_codes, cache.k_params,
+                                                cache.v_params)]
+    return type(cache)(1, cache.kv_heads, cache.head_dim, cache.capacity, cache.bits_k,
+                       cache.bits_v, cache.group,
+                       *[t[b * n:(b + 1) * n] for t, n in zip(
+                           (cache.k_codes, cache.v_codes, cache.k_params, cache.v_params), per)])
+
+
+def run_ours(args, rank, world, device):
+    w = workloads.WORKLOADS[args.workload]
+    bits = tuple(int(x) for x in args.bits.split(",")) if args.bits else w.bits[-1] \
+        if w.name == "long" else w.bits[0]
+    rotate = args.rotate
+    arm = Arm(w, bits, rotate, device)
+    stream = torch.cuda.current_stream()
+
+    # warm-up (also loads every kernel and the error-word address)
+    for i in range(max(args.warmup, 1)):
+        arm.step(i % rotate)
+    torch.cuda.synchronize()
+    flags = arm.kvq.kvq_device_error_flags()
+    if flags:
+        raise RuntimeError(f"device error flags {flags} during warm-up")
+
+    # one CUDA graph per rotation set
+    graphs = []
+    for r in range(rotate):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            arm.step(r)
+        graphs.append(g)
+    for i in range(args.warmup):
+        graphs[i % rotate].replay()
+    torch.cuda.synchronize()
+
+    # ---------------- timed region: exactly K steps
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device() if not os.environ.get("CUDA_VISIBLE_DEVICES")
+                      else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[
+                          torch.cuda.current_device()])) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            graphs[i % rotate].replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    flags = arm.kvq.kvq_device_error_flags()
+
+    nbytes = algorithmic_bytes(w, bits, arm.n_new, arm.read)
+    step_bytes = nbytes["quantize"] * (1 if arm.n_new else 0) + nbytes["decode"]
+
+    # ---------------- per-kernel durations (events inside a graph, GPU kept busy)
+    kern = per_kernel_times(arm, rotate, stream, reps=max(10, min(args.steps, 40)))
+    hbm_peak, peak_kind = peaks()
+    roof = {}
+    for name, key in (("quantize", "quantize"), ("decode_attention", "decode")):
+        if name not in kern:
+            continue
+        t_s = kern[name] / 1e3
+        ach = nbytes[key] / t_s / 1e9
+        roof[name] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak,
+                      "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
+                      "traffic": measured_traffic("quantize" if key == "quantize" else "decode",
+                                                  w.name),
+                      "ms": round(kern[name], 5), "algorithmic_bytes": nbytes[key],
+                      "peak_source": f"{peak_kind} hbm_gbs (copy)"}
+    dominant = "quantize" if "quantize" in roof and kern["quantize"] >= kern.get(
+        "decode_attention", 0) else "decode_attention"
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(arm, args, step_bytes, world, device)
+
+    result = {
+        "metric": METRIC,
+        "value": round(world * step_bytes / (ms_step / 1e3) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+            "head_dim": w.head_dim, "context": w.context, "input_dtype": w.dtype,
+            "bits_k": bits[0], "bits_v": bits[1], "group": w.group,
+            "step": ("quantize full cache + decode + combine" if w.name == "llama3_8b" else
+                     f"append {arm.n_new} + decode + combine"),
+            "split_tokens": arm.split_tokens,
+            "l2": f"{rotate} rotating input/cache sets (each step's data last touched "
+                  f"{rotate - 1} steps earlier), graph replay",
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+        },
+        "kv_tokens_per_s": round(world * nbytes["tokens"] / (ms_step / 1e3), 1),
+        "roofline": dict(roof[dominant], kernel=dominant),
+        "roofline_by_kernel": roof,
+        "gpu_launches": arm.launches_per_step * args.steps,
+        "device_error_flags": flags,
+        "e2e": e2e,
+        "clocks": clocks.summary(),
+        "arith": "binary32 quantizer; exact integer codes x binary16 operands on tensor "
+                 "cores with binary32 accumulation; binary32 softmax",
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, bits, args.cpu_seconds)
+    if world > 1:
+        for g in graphs:
+            del g
+    return result
+
+
+def per_kernel_times(arm, rotate, stream, reps):
+    """Average device time of the quantize launch and of the decode-attention
+    call (decode + combine), from events captured inside per-set graphs; a
+    sleep kernel keeps the GPU busy so that launch gaps are not timed."""
+    evs, graphs = [], []
+    for r in range(rotate):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            e[0].record()
+            arm.quantize(r)
+            e[1].record()
+            arm.decode(r)
+            e[2].record()
+        evs.append(e)
+        graphs.append(g)
+    q, d = [], []
+    for i in range(reps):
+        r = i % rotate
+        torch.cuda._sleep(200000)
+        graphs[r].replay()
+        torch.cuda.synchronize()
+        e = evs[r]
+        q.append(e[0].elapsed_time(e[1]))
+        d.append(e[1].elapsed_time(e[2]))
+    out = {"decode_attention": statistics.mean(d)}
+    if arm.n_new:
+        out["quantize"] = statistics.mean(q)
+    return out
+
+
+def run_e2e(arm, args, step_bytes, world, device):
+    """Same step through the public API with pinned host buffers: H2D of the
+    step's inputs, quantize + decode, D2H of the output, every step."""
+    s0 = arm.sets[0]
+    hk = s0["k"].cpu().pin_memory()
+    hv = s0["v"].cpu().pin_memory()
+    hq = s0["q"].cpu().pin_memory()
+    hout = torch.empty_like(s0["out"], device="cpu").pin_memory()
+    k_dev, v_dev, q_dev = torch.empty_like(s0["k"]), torch.empty_like(s0["v"]), torch.empty_like(s0["q"])
+    cache = s0["cache"]
+    stream = torch.cuda.current_stream()
+
+    def one():
+        k_dev.copy_(hk, non_blocking=True)
+        v_dev.copy_(hv, non_blocking=True)
+        q_dev.copy_(hq, non_blocking=True)
+        if arm.n_new:
+            arm.kvq.kvq_quantize_append(cache, k_dev, v_dev, arm.pos_t)
+        arm.kvq.kvq_decode_attention(cache, q_dev, arm.lens, arm.max_len, out=s0["out"],
+                                     workspace=arm.ws)
+        hout.copy_(s0["out"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 20))
+    if world > 1:
+        torch.distributed.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = (hk.numel() * hk.element_size() + hv.numel() * hv.element_size() +
+           hq.numel() * hq.element_size()) if arm.n_new else hq.numel() * hq.element_size()
+    return {"value": round(world * step_bytes / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 4), "steps": steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+
+
+# ---------------------------------------------------------- oracle (CPU)
+def oracle_step(w, bits, batch_rows, seed=0):
+    """One oracle pass (quantize + decode) over `batch_rows` batch rows of the
+    workload; returns (seconds, algorithmic bytes of that sample)."""
+    import oracle
+    n_new, pos, read = step_shape(w, bits)
+    ks, vs = workloads.make_kv(w, max(read[:batch_rows]), seed=seed, batch=batch_rows)
+    q = workloads.make_q(w, seed=seed, batch=batch_rows)
+    kb, dt = workloads.as_bits(ks)
+    vb, _ = workloads.as_bits(vs)
+    qb, _ = workloads.as_bits(q)
+    cap = (max(read[:batch_rows]) + 15) // 16 * 16
+    hc = oracle.HostCache(batch_rows, w.kv_heads, w.head_dim, cap, bits[0], bits[1], w.group)
+    t = time.perf_counter()
+    hc.quantize_append(kb, vb, [0] * batch_rows, dtype=dt)
+    hc.decode_attention(qb, w.q_heads, read[:batch_rows], q_dtype=dt)
+    sec = time.perf_counter() - t
+    nb = algorithmic_bytes(w, bits, max(read[:batch_rows]), read[:batch_rows])
+    scale = batch_rows / w.batch
+    # the oracle always quantizes the whole sample (a prefill), like the default step
+    return sec, (nb["quantize"] * batch_rows / w.batch + nb["decode"] * scale), sum(read[:batch_rows])
+
+
+def cpu_baseline(w, bits, budget_s):
+    import oracle
+    oracle.build()
+    total_s, total_b, total_t, runs = 0.0, 0.0, 0, 0
+    while total_s < budget_s or runs == 0:
+        s, b, t = oracle_step(w, bits, 1, seed=runs)
+        total_s += s
+        total_b += b
+        total_t += t
+        runs += 1
+    return {"value": round(total_b / total_s / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "kv_tokens_per_s": round(total_t / total_s, 1),
+            "sample": f"{runs} x one batch row of {w.name} (quantize its full context + decode "
+                      f"all its query heads), single-threaded C oracle, {total_s:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle as it stands, on a bounded sample per step."""
+    import oracle
+    oracle.build()
+    w = workloads.WORKLOADS[args.workload]
+    bits = w.bits[0]
+    for i in range(args.warmup):
+        oracle_step(w, bits, 1, seed=i)
+    tot_s, tot_b, tot_t = 0.0, 0.0, 0
+    for i in range(args.steps):
+        s, b, t = oracle_step(w, bits, 1, seed=i)
+        tot_s, tot_b, tot_t = tot_s + s, tot_b + b, tot_t + t
+    value = round(tot_b / tot_s / 1e9, 4)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tot_s / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads,
+                   "kv_heads": w.kv_heads, "head_dim": w.head_dim, "context": w.context,
+                   "bits_k": bits[0], "bits_v": bits[1], "group": w.group,
+                   "step": "one batch row of the workload per step (bounded sample)"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "one batch row per step, single-threaded C oracle"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "kv_tokens_per_s": round(tot_t / tot_s, 1),
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama3_8b", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--bits", default=None, help="bits_k,bits_v (default: the workload's)")
+    ap.add_argument("--rotate", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    try:
+        res = run_ours(args, rank, world, device)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,333 @@
+// Host side of the C ABI declared in kvq.h: argument validation, the
+// split-K plan, kernel selection and launches.  No allocation anywhere.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "internal.h"
+
+namespace kvq {
+bool get_decode_kernel_k2v2(int, int, int, DecodeKernel*);
+bool get_decode_kernel_k2v4(int, int, int, DecodeKernel*);
+bool get_decode_kernel_k2v8(int, int, int, DecodeKernel*);
+bool get_decode_kernel_k4v2(int, int, int, DecodeKernel*);
+bool get_decode_kernel_k4v4(int, int, int, DecodeKernel*);
+bool get_decode_kernel_k4v8(int, int, int, DecodeKernel*);
+bool get_decode_kernel_k8v2(int, int, int, DecodeKernel*);
+bool get_decode_kernel_k8v4(int, int, int, DecodeKernel*);
+bool get_decode_kernel_k8v8(int, int, int, DecodeKernel*);
+
+bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int num_groups, int variant,
+                       DecodeKernel* out) {
+  using Fn = bool (*)(int, int, int, DecodeKernel*);
+  static const Fn table[3][3] = {
+      {get_decode_kernel_k2v2, get_decode_kernel_k2v4, get_decode_kernel_k2v8},
+      {get_decode_kernel_k4v2, get_decode_kernel_k4v4, get_decode_kernel_k4v8},
+      {get_decode_kernel_k8v2, get_decode_kernel_k8v4, get_decode_kernel_k8v8}};
+  auto idx = [](int b) { return b == 2 ? 0 : b == 4 ? 1 : b == 8 ? 2 : -1; };
+  const int i = idx(bits_k), j = idx(bits_v);
+  if (i < 0 || j < 0) return false;
+  return table[i][j](head_dim, num_groups, variant, out);
+}
+}  // namespace kvq
+
+// Per-device error word (one copy on every device that loads the library).
+static __device__ uint32_t g_kvq_device_error;
+
+namespace {
+
+using kvq::DecodeKernel;
+
+constexpr int kMaxDevices = 64;
+
+int to_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_bits(int b) { return b == 2 || b == 4 || b == 8; }
+
+int check_shape(int B, int Hkv, int D, int cap, int bk, int bv, int G) {
+  if (B < 1 || Hkv < 1 || cap < 16 || cap % 16 != 0) return KVQ_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return KVQ_ERR_UNSUPPORTED;
+  if (!valid_bits(bk) || !valid_bits(bv)) return KVQ_ERR_UNSUPPORTED;
+  if (G != 32 && G != 64 && G != 128) return KVQ_ERR_UNSUPPORTED;
+  if (G > D) return KVQ_ERR_INVALID_ARG;
+  if (B > 65535 || Hkv > 65535) return KVQ_ERR_UNSUPPORTED;  // grid limits
+  return KVQ_OK;
+}
+
+int check_cache(const kvq_cache_desc* c) {
+  if (!c || c->reserved != 0) return KVQ_ERR_INVALID_ARG;
+  const int st = check_shape(c->batch, c->kv_heads, c->head_dim, c->capacity, c->bits_k,
+                             c->bits_v, c->group);
+  if (st != KVQ_OK) return st;
+  const void* ptrs[4] = {c->k_codes, c->v_codes, c->k_params, c->v_params};
+  for (const void* p : ptrs)
+    if (!p || !aligned(p, 16)) return KVQ_ERR_INVALID_ARG;
+  return KVQ_OK;
+}
+
+bool valid_dtype(int t) { return t == KVQ_F32 || t == KVQ_BF16 || t == KVQ_F16; }
+
+// Device address of the error word on the current device (looked up once per
+// device; the symbol's host-side name is not a device address).
+int error_word(uint32_t** out) {
+  static uint32_t* ptrs[kMaxDevices] = {};
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t status[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
+  std::call_once(once[dev], [dev] {
+    void* p = nullptr;
+    status[dev] = cudaGetSymbolAddress(&p, g_kvq_device_error);
+    ptrs[dev] = static_cast<uint32_t*>(p);
+  });
+  if (status[dev] != cudaSuccess) return KVQ_ERR_CUDA;
+  *out = ptrs[dev];
+  return KVQ_OK;
+}
+
+// Opt a kernel in to more than 48 KB of dynamic shared memory, once per
+// (device, kernel).
+cudaError_t prepare_kernel(const DecodeKernel& k) {
+  static std::mutex mu;
+  static std::set<std::pair<int, const void*>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({dev, k.fn})) return cudaSuccess;
+  e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem_bytes);
+  if (e == cudaSuccess) done.insert({dev, k.fn});
+  return e;
+}
+
+struct Plan {
+  int heads_per_cta, head_groups, split_tokens, num_splits;
+  size_t ws_bytes;
+};
+
+int variant_of(int heads_per_cta, int q_dtype) {
+  return (heads_per_cta <= 4 ? 0 : 2) + (q_dtype == KVQ_F32 ? 1 : 0);
+}
+
+// Split-K plan.  Tokens per split are a multiple of the 64-token stage.  The
+// grid aims at two waves of resident CTAs (load balance over ragged lengths)
+// while keeping at least 256 tokens per split (partial-result traffic).  It
+// depends only on the shape, Hq, max_seq_len and the device.
+int make_plan(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
+  const int gq = Hq / c->kv_heads;
+  p->heads_per_cta = gq < 8 ? gq : 8;
+  p->head_groups = (gq + p->heads_per_cta - 1) / p->heads_per_cta;
+  if (static_cast<long long>(c->kv_heads) * p->head_groups > 65535) return KVQ_ERR_UNSUPPORTED;
+  if (max_seq_len <= 0) {
+    p->split_tokens = 64;
+    p->num_splits = 0;
+    p->ws_bytes = 0;
+    return KVQ_OK;
+  }
+  DecodeKernel k;
+  if (!kvq::get_decode_kernel(c->head_dim, c->bits_k, c->bits_v, c->head_dim / c->group,
+                              variant_of(p->heads_per_cta, KVQ_BF16), &k))
+    return KVQ_ERR_UNSUPPORTED;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  if (prepare_kernel(k) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.fn, k.threads, k.smem_bytes) !=
+          cudaSuccess)
+    return KVQ_ERR_CUDA;
+  if (per_sm < 1) per_sm = 1;
+  const long long units = static_cast<long long>(c->batch) * c->kv_heads * p->head_groups;
+  const long long want = 2LL * sms * per_sm;
+  const long long max64 = (max_seq_len + 63LL) / 64 * 64;
+  long long split = (units * max_seq_len + want - 1) / want;
+  split = (split + 63) / 64 * 64;
+  if (split < 256) split = 256;
+  if (split > max64) split = max64;
+  if (const char* env = std::getenv("KVQ_SPLIT_TOKENS")) {
+    const long long v = std::atoll(env);
+    if (v >= 64 && v % 64 == 0) split = v;
+  }
+  p->split_tokens = static_cast<int>(split);
+  p->num_splits = static_cast<int>((max_seq_len + split - 1) / split);
+  if (p->num_splits > 65535) return KVQ_ERR_UNSUPPORTED;
+  p->ws_bytes = static_cast<size_t>(c->batch) * Hq * p->num_splits * (c->head_dim + 1) * 4;
+  p->ws_bytes = (p->ws_bytes + 15) / 16 * 16;
+  return KVQ_OK;
+}
+
+int check_decode_args(const kvq_cache_desc* c, int Hq, int max_seq_len) {
+  const int st = check_cache(c);
+  if (st != KVQ_OK) return st;
+  if (Hq < 1 || Hq % c->kv_heads != 0 || max_seq_len < 0) return KVQ_ERR_INVALID_ARG;
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvq_cache_bytes(int32_t batch, int32_t kv_heads, int32_t head_dim, int32_t capacity,
+                       int32_t bits_k, int32_t bits_v, int32_t group, int32_t which) {
+  if (check_shape(batch, kv_heads, head_dim, capacity, bits_k, bits_v, group) != KVQ_OK) return 0;
+  const size_t slots = static_cast<size_t>(batch) * kv_heads;
+  switch (which) {
+    case KVQ_K_CODES: return slots * capacity * head_dim * bits_k / 8;
+    case KVQ_V_CODES: return slots * capacity * head_dim * bits_v / 8;
+    case KVQ_K_PARAMS:
+    case KVQ_V_PARAMS: return slots * capacity * (head_dim / group) * 4;
+    default: return 0;
+  }
+}
+
+int kvq_validate_cache(const kvq_cache_desc* cache) { return check_cache(cache); }
+
+int kvq_quantize_append(const kvq_cache_desc* cache, const void* k, const void* v,
+                        int32_t in_dtype, const int32_t* pos, int32_t n_new,
+                        kvq_stream_t stream) {
+  int st = check_cache(cache);
+  if (st != KVQ_OK) return st;
+  if (!valid_dtype(in_dtype) || n_new < 0 || n_new > cache->capacity) return KVQ_ERR_INVALID_ARG;
+  if (!k || !v || !pos || !aligned(k, 16) || !aligned(v, 16) || !aligned(pos, 4))
+    return KVQ_ERR_INVALID_ARG;
+  if (n_new == 0) return KVQ_OK;
+  kvq::QuantizeArgs a;
+  a.k = k;
+  a.v = v;
+  a.in_dtype = in_dtype;
+  a.k_codes = cache->k_codes;
+  a.v_codes = cache->v_codes;
+  a.k_params = static_cast<uint32_t*>(cache->k_params);
+  a.v_params = static_cast<uint32_t*>(cache->v_params);
+  a.pos = pos;
+  a.n_new = n_new;
+  a.batch = cache->batch;
+  a.kv_heads = cache->kv_heads;
+  a.head_dim = cache->head_dim;
+  a.capacity = cache->capacity;
+  a.bits_k = cache->bits_k;
+  a.bits_v = cache->bits_v;
+  a.group = cache->group;
+  st = error_word(&a.err);
+  if (st != KVQ_OK) return st;
+  return to_status(kvq::launch_quantize_append(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t kvq_decode_workspace_bytes(const kvq_cache_desc* cache, int32_t num_q_heads,
+                                  int32_t max_seq_len) {
+  if (check_decode_args(cache, num_q_heads, max_seq_len) != KVQ_OK) return 0;
+  Plan p;
+  if (make_plan(cache, num_q_heads, max_seq_len, &p) != KVQ_OK) return 0;
+  return p.ws_bytes;
+}
+
+int32_t kvq_decode_split_tokens(const kvq_cache_desc* cache, int32_t num_q_heads,
+                                int32_t max_seq_len) {
+  if (check_decode_args(cache, num_q_heads, max_seq_len) != KVQ_OK) return 0;
+  Plan p;
+  if (make_plan(cache, num_q_heads, max_seq_len, &p) != KVQ_OK) return 0;
+  return p.split_tokens;
+}
+
+int kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int32_t q_dtype,
+                         int32_t num_q_heads, const int32_t* seq_lens, int32_t max_seq_len,
+                         float sm_scale, void* out, int32_t out_dtype, void* workspace,
+                         size_t workspace_bytes, kvq_stream_t stream) {
+  int st = check_decode_args(cache, num_q_heads, max_seq_len);
+  if (st != KVQ_OK) return st;
+  if (!valid_dtype(q_dtype) || !valid_dtype(out_dtype)) return KVQ_ERR_INVALID_ARG;
+  if (!q || !seq_lens || !out || !aligned(q, 16) || !aligned(seq_lens, 4) || !aligned(out, 16))
+    return KVQ_ERR_INVALID_ARG;
+  if (!(sm_scale == sm_scale)) return KVQ_ERR_INVALID_ARG;  // NaN
+  Plan p;
+  st = make_plan(cache, num_q_heads, max_seq_len, &p);
+  if (st != KVQ_OK) return st;
+  if (p.ws_bytes > 0 && (!workspace || !aligned(workspace, 16) || workspace_bytes < p.ws_bytes))
+    return KVQ_ERR_WORKSPACE;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int D = cache->head_dim;
+  const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf(static_cast<float>(D));
+  float* ws_o = static_cast<float*>(workspace);
+  float* ws_lse = ws_o ? ws_o + static_cast<size_t>(cache->batch) * num_q_heads * p.num_splits * D
+                       : nullptr;
+  if (p.num_splits > 0) {
+    DecodeKernel k;
+    if (!kvq::get_decode_kernel(D, cache->bits_k, cache->bits_v, D / cache->group,
+                                variant_of(p.heads_per_cta, q_dtype), &k))
+      return KVQ_ERR_UNSUPPORTED;
+    if (prepare_kernel(k) != cudaSuccess) return KVQ_ERR_CUDA;
+    kvq::DecodeArgs a;
+    a.k_codes = cache->k_codes;
+    a.v_codes = cache->v_codes;
+    a.k_params = static_cast<const uint32_t*>(cache->k_params);
+    a.v_params = static_cast<const uint32_t*>(cache->v_params);
+    a.q = q;
+    a.q_dtype = q_dtype;
+    a.seq_lens = seq_lens;
+    a.batch = cache->batch;
+    a.kv_heads = cache->kv_heads;
+    a.q_heads = num_q_heads;
+    a.gq = num_q_heads / cache->kv_heads;
+    a.capacity = cache->capacity;
+    a.max_seq_len = max_seq_len;
+    a.heads_per_cta = p.heads_per_cta;
+    a.head_groups = p.head_groups;
+    a.split_tokens = p.split_tokens;
+    a.num_splits = p.num_splits;
+    a.sm_scale_log2 = scale * 1.4426950408889634f;
+    a.ws_o = ws_o;
+    a.ws_lse = ws_lse;
+    st = error_word(&a.err);
+    if (st != KVQ_OK) return st;
+    const dim3 grid(p.num_splits, cache->kv_heads * p.head_groups, cache->batch);
+    if (k.launch(a, grid, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  }
+  kvq::CombineArgs ca;
+  ca.ws_o = ws_o;
+  ca.ws_lse = ws_lse;
+  ca.seq_lens = seq_lens;
+  ca.out = out;
+  ca.out_dtype = out_dtype;
+  ca.batch = cache->batch;
+  ca.q_heads = num_q_heads;
+  ca.head_dim = D;
+  ca.capacity = cache->capacity;
+  ca.max_seq_len = max_seq_len;
+  ca.split_tokens = p.split_tokens;
+  ca.num_splits = p.num_splits;
+  return to_status(kvq::launch_combine(ca, s));
+}
+
+int kvq_device_error_flags(kvq_stream_t stream, uint32_t* flags) {
+  if (!flags) return KVQ_ERR_INVALID_ARG;
+  uint32_t* word = nullptr;
+  int st = error_word(&word);
+  if (st != KVQ_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, word, sizeof host, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, sizeof host, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  *flags = host;
+  return KVQ_OK;
+}
+
+const char* kvq_strerror(int32_t status) {
+  switch (status) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case KVQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case KVQ_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

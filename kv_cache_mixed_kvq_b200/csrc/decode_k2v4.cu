@@ -1,0 +1,8 @@
+// Decode kernel instances for keys at 2 bits and values at 4 bits.
+#include "decode.cuh"
+
+namespace kvq {
+bool get_decode_kernel_k2v4(int head_dim, int num_groups, int variant, DecodeKernel* out) {
+  return get_decode_kernel_bits<2, 4>(head_dim, num_groups, variant, out);
+}
+}  // namespace kvq

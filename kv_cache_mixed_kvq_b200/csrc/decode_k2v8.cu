@@ -1,0 +1,8 @@
+// Decode kernel instances for keys at 2 bits and values at 8 bits.
+#include "decode.cuh"
+
+namespace kvq {
+bool get_decode_kernel_k2v8(int head_dim, int num_groups, int variant, DecodeKernel* out) {
+  return get_decode_kernel_bits<2, 8>(head_dim, num_groups, variant, out);
+}
+}  // namespace kvq

@@ -1,0 +1,8 @@
+// Decode kernel instances for keys at 8 bits and values at 8 bits.
+#include "decode.cuh"
+
+namespace kvq {
+bool get_decode_kernel_k8v8(int head_dim, int num_groups, int variant, DecodeKernel* out) {
+  return get_decode_kernel_bits<8, 8>(head_dim, num_groups, variant, out);
+}
+}  // namespace kvq

@@ -1,0 +1,72 @@
+// Declarations shared by the host entry points and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+struct QuantizeArgs {
+  const void* k;
+  const void* v;
+  int in_dtype;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  uint32_t* k_params;  // binary16 (scale, zero) pairs
+  uint32_t* v_params;
+  const int32_t* pos;
+  int n_new;
+  int batch, kv_heads, head_dim, capacity, bits_k, bits_v, group;
+  uint32_t* err;
+};
+
+cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream);
+
+// Split-K decode.  One CTA = one (split, kv head x head group, batch row).
+struct DecodeArgs {
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const uint32_t* k_params;
+  const uint32_t* v_params;
+  const void* q;
+  int q_dtype;
+  const int32_t* seq_lens;
+  int batch, kv_heads, q_heads, gq, capacity, max_seq_len;
+  int heads_per_cta;  // <= 8
+  int head_groups;    // ceil(gq / heads_per_cta)
+  int split_tokens;   // multiple of 64
+  int num_splits;     // grid.x
+  float sm_scale_log2;  // softmax scale times log2(e)
+  float* ws_o;        // [B][Hq][num_splits][D] partial outputs
+  float* ws_lse;      // [B][Hq][num_splits] log2-domain log-sum-exp
+  uint32_t* err;
+};
+
+// Kernel variant, from the query type and the number of heads per CTA:
+//   0: 16-bit Q, <= 4 heads    1: fp32 Q, <= 4 heads
+//   2: 16-bit Q, 5..8 heads    3: fp32 Q, 5..8 heads
+struct DecodeKernel {
+  const void* fn;      // __global__ function
+  int threads;
+  int smem_bytes;
+  cudaError_t (*launch)(const DecodeArgs&, dim3 grid, cudaStream_t stream);
+};
+
+// Returns false if (D, bits_k, bits_v, groups, variant) has no instance.
+bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int num_groups, int variant,
+                       DecodeKernel* out);
+
+struct CombineArgs {
+  const float* ws_o;
+  const float* ws_lse;
+  const int32_t* seq_lens;
+  void* out;
+  int out_dtype;
+  int batch, q_heads, head_dim, capacity, max_seq_len, split_tokens, num_splits;
+};
+
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+
+}  // namespace kvq
