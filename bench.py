@@ -335,7 +335,7 @@ def per_kernel_times(arm, rotate, stream, reps):
     sleep kernel keeps the GPU busy so that launch gaps are not timed."""
     evs, graphs = [], []
     for r in range(rotate):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             e[0].record()

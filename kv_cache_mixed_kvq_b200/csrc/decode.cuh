@@ -184,6 +184,9 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   float m_run[HT], l_run[HT];
   float oacc[KSTEPS][NP][4];
   float zacc[NP][NG];
+  // Power-of-two exponent applied to the output weights p * scale_v so that
+  // their binary16 parts stay normal; only ever decreases (see below).
+  int u_run = 100;
 #pragma unroll
   for (int hs = 0; hs < HT; ++hs) {
     m_run[hs] = -INFINITY;
@@ -355,14 +358,35 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         __syncwarp();
         changed = __any_sync(0xffffffffu, changed);
 
-        // ---- weights p * scale_v as binary16 high/low parts (B operand)
+        // ---- weights p * scale_v as binary16 high/low parts (B operand).
+        // They are scaled by 2^u_run with u_run chosen from the largest value
+        // scale in the tile (p <= 1), so that the largest weight stays below
+        // 2^15 and the low part of every weight that matters stays a normal
+        // binary16.  When a tile needs a smaller exponent, the output
+        // accumulators are rescaled by the (exact) power of two.
+        const int kk[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
+        float2 svz[4][NG];
+        float smax = 0.0f;
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int gr = 0; gr < NG; ++gr) {
+            svz[x][gr] = unpack_half2(vp[kk[x] * NG + gr]);
+            if (kk[x] < nvalid) smax = fmaxf(smax, svz[x][gr].x);
+          }
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 1));
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 2));
+        const int u_need = smax > 0.0f ? min(100, 14 - ilogbf(smax)) : 100;
+        const bool u_changed = u_need < u_run;
+        const float u_shift = u_changed ? __int_as_float((127 + u_need - u_run) << 23) : 1.0f;
+        if (u_changed) u_run = u_need;
+        const float f_u = __int_as_float((127 + u_run) << 23);
         uint32_t bp[NP][NG][2];
 #pragma unroll
         for (int pt = 0; pt < NP; ++pt) {
           const int hd = 4 * pt + (g >> 1);
           const int part = g & 1;
           float pv[4];
-          int kk[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
 #pragma unroll
           for (int x = 0; x < 4; ++x) pv[x] = wpex[kk[x] * 8 + hd];
           const float az = changed ? walph[hd] : 1.0f;
@@ -372,21 +396,20 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
             float z = 0.0f;
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
-              const float2 sz = unpack_half2(vp[kk[x] * NG + gr]);
-              const float P = pv[x] == 0.0f ? 0.0f : pv[x] * sz.x;
+              const float P = pv[x] == 0.0f ? 0.0f : (pv[x] * f_u) * svz[x][gr].x;
               const __half hi = __float2half_rn(P);
               hv[x] = part ? __float2half_rn(P - __half2float(hi)) : hi;
-              z += pv[x] == 0.0f ? 0.0f : pv[x] * sz.y;
+              z += pv[x] == 0.0f ? 0.0f : pv[x] * svz[x][gr].y;
             }
             bp[pt][gr][0] = pack_half2(hv[0], hv[1]);
             bp[pt][gr][1] = pack_half2(hv[2], hv[3]);
             if (part == 0) zacc[pt][gr] = fmaf(zacc[pt][gr], az, z);
           }
         }
-        if (changed) {
+        if (changed || u_changed) {
 #pragma unroll
           for (int pt = 0; pt < NP; ++pt) {
-            const float ao = walph[4 * pt + c];
+            const float ao = (changed ? walph[4 * pt + c] : 1.0f) * u_shift;
 #pragma unroll
             for (int j = 0; j < KSTEPS; ++j)
 #pragma unroll
@@ -450,8 +473,8 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       const int head = 4 * pt + c;
 #pragma unroll
       for (int j = 0; j < KSTEPS; ++j) {
-        const float s0 = ldexpf(1.0f, 24 - field_pos<C::BV>((2 * j) % (16 / C::BV)));
-        const float s1 = ldexpf(1.0f, 24 - field_pos<C::BV>((2 * j + 1) % (16 / C::BV)));
+        const float s0 = ldexpf(1.0f, 24 - u_run - field_pos<C::BV>((2 * j) % (16 / C::BV)));
+        const float s1 = ldexpf(1.0f, 24 - u_run - field_pos<C::BV>((2 * j + 1) % (16 / C::BV)));
         ob[(warp * 8 + head) * D + 16 * j + g] = (oacc[j][pt][0] + oacc[j][pt][1]) * s0;
         ob[(warp * 8 + head) * D + 16 * j + 8 + g] = (oacc[j][pt][2] + oacc[j][pt][3]) * s1;
       }

@@ -110,8 +110,13 @@ def test_split_count_invariance(ora):
         out, ref = _run(ora, 2, 2, 8, 128, 4, 2, 64, [1000, 613], seed=11, split_tokens=st)
         compare_attention(out, ref)
         outs.append(out.cpu().numpy())
+    # Splits change the order of the sums and the softmax reference maxima;
+    # the tensor cores truncate products of binary16 subnormal operands to
+    # about 2^-19.6 of the sum of |terms| per instruction (measured), so the
+    # outputs of different split counts agree to ~1e-4, far inside the 2e-3
+    # bar, while a wrong log-sum-exp weight would move them by O(0.1).
     for o in outs[1:]:
-        assert np.allclose(o, outs[0], rtol=1e-5, atol=1e-6)
+        assert np.abs(o - outs[0]).max() <= 2e-4
 
 
 def test_sm_scale_and_peaked_softmax(ora):
