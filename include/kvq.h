@@ -231,6 +231,37 @@ int kvq_decode_attention(const kvq_cache_desc* cache, const void* q,
                          kvq_stream_t stream);
 
 /*
+ * Size of the fixed device scratch array used by
+ * kvq_decode_attention_static(): 4 MiB, held on every device that loads the
+ * library until the process exits.
+ */
+#define KVQ_STATIC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * kvq_decode_attention() for callers that cannot allocate device memory.
+ * The summary page has no counterpart to this call; it exists for engines
+ * that must not call cudaMalloc on the request path (it can synchronize the
+ * device and fail under fragmentation) and for plain-C hosts without a
+ * device allocator.  Arguments as for kvq_decode_attention(), minus the
+ * workspace: the split-K partial results go to a fixed array of
+ * KVQ_STATIC_SCRATCH_BYTES inside the library's device image.
+ *   - Returns KVQ_ERR_WORKSPACE, launching nothing, when this shape needs
+ *     more scratch than that (kvq_decode_workspace_bytes() tells how much).
+ *   - Allocates nothing.  The first call on each device looks up the array's
+ *     device address (cudaGetSymbolAddress) with that device current; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents; nothing in it needs to start at zero.  Calls whose kernels
+ *     may overlap on the GPU (different streams without ordering between
+ *     them) race on the array: serialize them.
+ */
+int kvq_decode_attention_static(const kvq_cache_desc* cache, const void* q,
+                                int32_t q_dtype, int32_t num_q_heads,
+                                const int32_t* seq_lens, int32_t max_seq_len,
+                                float sm_scale, void* out, int32_t out_dtype,
+                                kvq_stream_t stream);
+
+/*
  * Tokens per split that kvq_decode_attention() will use for these
  * arguments on the current device (0 if invalid).  Informational.
  */
