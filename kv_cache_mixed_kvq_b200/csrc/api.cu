@@ -5,7 +5,9 @@
 #include <cmath>
 #include <cstdlib>
 #include <mutex>
+#include <map>
 #include <set>
+#include <tuple>
 #include <utility>
 
 #include "internal.h"
@@ -115,11 +117,14 @@ int variant_of(int heads_per_cta, int q_dtype) {
   return (heads_per_cta <= 4 ? 0 : 2) + (q_dtype == KVQ_F32 ? 1 : 0);
 }
 
-// Split-K plan.  Tokens per split are a multiple of the 64-token stage.  The
-// grid aims at two waves of resident CTAs (load balance over ragged lengths)
-// while keeping at least 256 tokens per split (partial-result traffic).  It
-// depends only on the shape, Hq, max_seq_len and the device.
-int make_plan(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
+// Split-K plan.  Tokens per split are a multiple of the 64-token stage.
+// When one wave of resident CTAs can cover every (batch row, kv head) with
+// splits of at least 256 tokens, use exactly one wave (equal lengths finish
+// together, nothing waits for a second wave).  Otherwise aim at about four
+// waves, so that the block scheduler can balance ragged lengths, with at
+// least 256 tokens per split (partial-result traffic).  The plan depends
+// only on the shape, Hq, max_seq_len and the device.
+int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
   const int gq = Hq / c->kv_heads;
   p->heads_per_cta = gq < 8 ? gq : 8;
   p->head_groups = (gq + p->heads_per_cta - 1) / p->heads_per_cta;
@@ -144,10 +149,17 @@ int make_plan(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
     return KVQ_ERR_CUDA;
   if (per_sm < 1) per_sm = 1;
   const long long units = static_cast<long long>(c->batch) * c->kv_heads * p->head_groups;
-  const long long want = 2LL * sms * per_sm;
+  const long long slots = static_cast<long long>(sms) * per_sm;
   const long long max64 = (max_seq_len + 63LL) / 64 * 64;
-  long long split = (units * max_seq_len + want - 1) / want;
-  split = (split + 63) / 64 * 64;
+  long long split = 0;
+  if (units <= slots) {
+    const long long per_unit = slots / units;
+    split = ((max_seq_len + per_unit - 1) / per_unit + 63) / 64 * 64;
+  }
+  if (split < 256) {
+    const long long want = 4 * slots;
+    split = ((units * max_seq_len + want - 1) / want + 63) / 64 * 64;
+  }
   if (split < 256) split = 256;
   if (split > max64) split = max64;
   if (const char* env = std::getenv("KVQ_SPLIT_TOKENS")) {
@@ -160,6 +172,35 @@ int make_plan(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
   p->ws_bytes = static_cast<size_t>(c->batch) * Hq * p->num_splits * (c->head_dim + 1) * 4;
   p->ws_bytes = (p->ws_bytes + 15) / 16 * 16;
   return KVQ_OK;
+}
+
+// Plans are cached per (device, shape, Hq, max_seq_len, split override):
+// the occupancy query behind a plan costs microseconds of host time.
+int make_plan(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
+  using Key = std::tuple<int, int, int, int, int, int, int, int, int, int, long long>;
+  static std::mutex mu;
+  static std::map<Key, Plan> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
+  long long override_split = 0;
+  if (const char* env = std::getenv("KVQ_SPLIT_TOKENS")) override_split = std::atoll(env);
+  const Key key{dev, c->batch, c->kv_heads, c->head_dim, c->bits_k, c->bits_v, c->group, Hq,
+                max_seq_len, c->capacity, override_split};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *p = it->second;
+      return KVQ_OK;
+    }
+  }
+  const int st = make_plan_uncached(c, Hq, max_seq_len, p);
+  if (st == KVQ_OK) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() > 4096) cache.clear();
+    cache.emplace(key, *p);
+  }
+  return st;
 }
 
 int check_decode_args(const kvq_cache_desc* c, int Hq, int max_seq_len) {

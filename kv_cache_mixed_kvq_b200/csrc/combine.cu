@@ -22,6 +22,9 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
   const int ns = (len + a.split_tokens - 1) / a.split_tokens;
   const size_t base = static_cast<size_t>(row) * a.num_splits;
 
+  // weights 2^(lse_s - L): lanes load the log-sum-exps of 32 splits at a
+  // time in parallel; the partial outputs are then read with the loads of
+  // several splits in flight.
   float L = -INFINITY;
   for (int s = lane; s < ns; s += 32) L = fmaxf(L, a.ws_lse[base + s]);
 #pragma unroll
@@ -31,20 +34,33 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
   float den = 0.0f;
-  for (int s = 0; s < ns; ++s) {
-    const float w = exp2f(a.ws_lse[base + s] - L);
-    den += w;
-    const float* o = a.ws_o + (base + s) * D + lane * PER;
-    if constexpr (PER == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(o);
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
-      acc[2] = fmaf(w, v.z, acc[2]);
-      acc[3] = fmaf(w, v.w, acc[3]);
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(o);
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const int cnt = min(32, ns - s0);
+    const float wl = lane < cnt ? exp2_approx(a.ws_lse[base + s0 + lane] - L) : 0.0f;
+    constexpr int U = 4;
+    for (int s = 0; s < cnt; s += U) {
+      float w[U];
+      float v[U][PER];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        w[u] = __shfl_sync(0xffffffffu, wl, (s + u) & 31);
+        const int si = s0 + min(s + u, cnt - 1);
+        const float* o = a.ws_o + (base + si) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 t = *reinterpret_cast<const float4*>(o);
+          v[u][0] = t.x; v[u][1] = t.y; v[u][2] = t.z; v[u][3] = t.w;
+        } else {
+          const float2 t = *reinterpret_cast<const float2*>(o);
+          v[u][0] = t.x; v[u][1] = t.y;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (s + u >= cnt) break;
+        den += w[u];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) acc[i] = fmaf(w[u], v[u][i], acc[i]);
+      }
     }
   }
   const float inv = ns > 0 ? 1.0f / den : 0.0f;

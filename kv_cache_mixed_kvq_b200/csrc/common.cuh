@@ -95,14 +95,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
       : "memory");
 }
 
+// Test for the completion of the phase with the given parity; the thread may
+// be suspended (up to the hint, in nanoseconds) until it completes, so that
+// waiting warps do not spin on the issue slots.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
@@ -116,10 +119,8 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // Longest a pipeline wait may take before the kernel gives up (1 s).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
-// Bounded wait on an mbarrier phase: returns false (and flags
-// KVQ_DEVERR_TIMEOUT) if the phase did not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* err) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait_bounded: keep waiting, up to kWaitLimitNs.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* err) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -128,6 +129,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
       return false;
     }
   }
+}
+
+// Bounded wait on an mbarrier phase: returns false (and flags
+// KVQ_DEVERR_TIMEOUT) if the phase did not complete within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, err);
 }
 
 // 1-D bulk copy global -> shared (no multicast), completion counted in bytes
@@ -150,6 +158,25 @@ __device__ __forceinline__ void mma_f16_16816(float d[4], uint32_t a0, uint32_t 
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 2^e as a binary32 value, for e in [-126, 127] (exact).
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// 2^x, hardware approximation (relative error ~2^-22; results below 2^-126
+// flush to zero), for softmax weights.
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two binary32 values rounded to binary16 (nearest even) in one register:
+// lo in bits 0..15, hi in bits 16..31.
+__device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {

@@ -17,25 +17,30 @@
 //    applied afterwards:  q.k^ = sum_g scale_g (q . c_g) + zero_g sum_{d in g} q_d
 //    and  o = sum_t (p_t scale_t) c_t + sum_t p_t zero_t;
 //  * the query (B operand of the score product) is scaled by a power of two
-//    and, for binary32 queries, split into binary16 high and low parts in two
-//    columns; the weights p_t * scale_t (B operand of the output product) are
-//    always split into high and low parts, so products keep ~22 bits;
-//  * online softmax in binary32 (exp2 domain), partial results per split are
-//    merged by a separate log-sum-exp combine kernel.
+//    and split into binary16 high and low parts in two columns (the low part
+//    is zero for 16-bit queries); the weights p_t * scale_t (B operand of the
+//    output product) are split the same way and scaled per warp by a power of
+//    two, so products keep ~22 bits;
+//  * online softmax in binary32 (exp2 domain) with a lazily updated maximum;
+//    partial results per split are merged by a separate log-sum-exp combine.
 #pragma once
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
 
 namespace kvq {
 
+// QS == 2: each lane's two score columns are the high and low parts of one
+// head (up to 4 heads per n-tile); QS == 1: two heads (up to 8 per n-tile).
 template <int D_, int BK_, int BV_, int NG_, int QS_, int NQ_, int NP_>
 struct DecodeCfg {
   static constexpr int D = D_, BK = BK_, BV = BV_, NG = NG_, QS = QS_, NQ = NQ_, NP = NP_;
   static constexpr int kWarps = 4;  // consumer warps
   static constexpr int kThreads = 32 * (kWarps + 1);
-  static constexpr int kStageTokens = 16 * kWarps;
-  static constexpr int kStages = 4;
+  static constexpr int TPW = 2;     // 16-token tiles per warp per stage
+  static constexpr int kStageTokens = 16 * TPW * kWarps;
   static constexpr int G = D / NG;
   static constexpr int KSTEPS = D / 16;  // k-steps (scores) == m-tiles (output)
   static constexpr int KROW = D * BK / 8;
@@ -48,14 +53,20 @@ struct DecodeCfg {
   static constexpr int WV = D * BV / 128;  // V words per half-lane
   static constexpr int PROW = NG * 4;
   static constexpr int STAGE_K = kStageTokens * KROW;
-  static constexpr int STAGE_V = kWarps * VTILE;
+  static constexpr int STAGE_V = TPW * kWarps * VTILE;
   static constexpr int STAGE_P = kStageTokens * PROW;
   static constexpr int STAGE_BYTES = STAGE_K + STAGE_V + 2 * STAGE_P;
+  static constexpr int kStages = STAGE_BYTES > 20000 ? 3 : 4;
   static constexpr int RING_BYTES = kStages * STAGE_BYTES;
-  static constexpr int PEX_FLOATS = kWarps * 16 * 8;
+  // staged output weights: per warp [group][head][part][WB_RS halves]
+  static constexpr int WB_RS = 24;  // halves per row: 16 positions + pad (conflict-free)
+  static constexpr int WB_HALVES = NG * 8 * 2 * WB_RS;
+  static constexpr int WB_BYTES = TPW * kWarps * WB_HALVES * 2;
   static constexpr int ALPHA_FLOATS = kWarps * 8;
-  static constexpr int SMEM_BYTES = RING_BYTES + 4 * (PEX_FLOATS + ALPHA_FLOATS) + 16 * kStages;
-  static constexpr int HT = QS == 1 ? 2 * NQ : NQ;  // score head slots per thread
+  static constexpr int MERGE_FLOATS = kWarps * 8 * (2 + NG) + 2 * 8 * (kWarps + 1);
+  static constexpr int SMEM_BYTES =
+      RING_BYTES + WB_BYTES + 4 * (ALPHA_FLOATS + MERGE_FLOATS) + 16 * kStages;
+  static constexpr int HT = QS == 1 ? 2 * NQ : NQ;  // score head slots per lane
   static_assert(RING_BYTES >= kWarps * 8 * D * 4, "merge buffer must fit in the ring");
   static_assert(STAGE_BYTES % 16 == 0 && STAGE_K % 16 == 0 && STAGE_V % 16 == 0, "alignment");
   static_assert(G >= 16 && G % 16 == 0, "group must cover whole 16-element steps");
@@ -105,14 +116,53 @@ __device__ __forceinline__ float warp_max_xor(float v, int lo_mask) {
   return v;
 }
 
+// (scale_a, scale_b) and (zero_a, zero_b) of two (scale, zero) binary16 pairs.
+__device__ __forceinline__ float2 scales_of(uint32_t a, uint32_t b) {
+  return unpack_half2(__byte_perm(a, b, 0x5410));
+}
+__device__ __forceinline__ float2 zeros_of(uint32_t a, uint32_t b) {
+  return unpack_half2(__byte_perm(a, b, 0x7632));
+}
+
+// D = A * B (C = 0), m16n8k16, fp16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_f16_16816_zc(float d[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                 uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// (scale, zero) words of two consecutive positions (N groups each).
+template <int N>
+__device__ __forceinline__ void lds_param_pair(const uint32_t* p, uint32_t (&w0)[N], uint32_t (&w1)[N]) {
+  if constexpr (N == 1) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    w0[0] = u.x;
+    w1[0] = u.y;
+  } else if constexpr (N == 2) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    w0[0] = u.x; w0[1] = u.y;
+    w1[0] = u.z; w1[1] = u.w;
+  } else {
+    static_assert(N == 4, "groups per row");
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint4 v = *reinterpret_cast<const uint4*>(p + 4);
+    w0[0] = u.x; w0[1] = u.y; w0[2] = u.z; w0[3] = u.w;
+    w1[0] = v.x; w1[1] = v.y; w1[2] = v.z; w1[3] = v.w;
+  }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a) {
   constexpr int D = C::D, NG = C::NG, NQ = C::NQ, NP = C::NP, QS = C::QS, HT = C::HT;
   constexpr int KSTEPS = C::KSTEPS, G = C::G;
   extern __shared__ __align__(128) uint8_t smem[];
-  float* pex = reinterpret_cast<float*>(smem + C::RING_BYTES);  // [warp][16 tokens][8 heads]
-  float* alph = pex + C::PEX_FLOATS;                            // [warp][8 heads]
-  uint64_t* full = reinterpret_cast<uint64_t*>(alph + C::ALPHA_FLOATS);
+  uint16_t* wbuf = reinterpret_cast<uint16_t*>(smem + C::RING_BYTES);  // staged weights
+  float* alph = reinterpret_cast<float*>(smem + C::RING_BYTES + C::WB_BYTES);  // [warp][8]
+  float* mrg = alph + C::ALPHA_FLOATS;                                     // merge area
+  uint64_t* full = reinterpret_cast<uint64_t*>(mrg + C::MERGE_FLOATS);
   uint64_t* empty = full + C::kStages;
 
   const int split = blockIdx.x;
@@ -183,10 +233,11 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   const int g = lane >> 2, c = lane & 3;
   float m_run[HT], l_run[HT];
   float oacc[KSTEPS][NP][4];
-  float zacc[NP][NG];
+  float2 zacc[HT][NG];  // zero term, score layout: (row g, row g+8) partials
   // Power-of-two exponent applied to the output weights p * scale_v so that
   // their binary16 parts stay normal; only ever decreases (see below).
   int u_run = 100;
+  float u_bound = pow2i(7 - 100);  // value scales below this keep the weights < 2^15
 #pragma unroll
   for (int hs = 0; hs < HT; ++hs) {
     m_run[hs] = -INFINITY;
@@ -199,9 +250,9 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
 #pragma unroll
       for (int r = 0; r < 4; ++r) oacc[j][pt][r] = 0.0f;
 #pragma unroll
-  for (int pt = 0; pt < NP; ++pt)
+  for (int hs = 0; hs < HT; ++hs)
 #pragma unroll
-    for (int gr = 0; gr < NG; ++gr) zacc[pt][gr] = 0.0f;
+    for (int gr = 0; gr < NG; ++gr) zacc[hs][gr] = make_float2(0.0f, 0.0f);
 
   if (warp < C::kWarps) {
     // -------- query fragments (B operand of the score product), once per CTA
@@ -211,17 +262,27 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     for (int nt = 0; nt < NQ; ++nt) {
       const int n = 8 * nt + g;
       const int head = QS == 2 ? n / 2 : n;
+      const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * D;
 #pragma unroll
       for (int j = 0; j < KSTEPS; ++j)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int d = 16 * j + 2 * c + (r & 1) + 8 * (r >> 1);
-          float v = 0.0f;
-          if (head < nh)
-            v = load_elem(a.q, a.q_dtype,
-                          (static_cast<size_t>(b) * a.q_heads + head0 + head) * D + d);
-          qraw[nt][j][r] = v;
-          amax = fmaxf(amax, fabsf(v));
+        for (int r = 0; r < 2; ++r) {
+          // elements d, d+1 with d = 16j + 2c + 8r
+          const size_t d = row + 16 * j + 2 * c + 8 * r;
+          float2 v = make_float2(0.0f, 0.0f);
+          if (head < nh) {
+            if (a.q_dtype == KVQ_F32) {
+              v = __ldg(reinterpret_cast<const float2*>(a.q) + d / 2);
+            } else {
+              const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(a.q) + d / 2);
+              v = a.q_dtype == KVQ_BF16
+                      ? make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u))
+                      : unpack_half2(u);
+            }
+          }
+          qraw[nt][j][2 * r] = v.x;
+          qraw[nt][j][2 * r + 1] = v.y;
+          amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
         }
     }
     amax = warp_max_xor(amax, 1);
@@ -229,275 +290,399 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     uint32_t bq[NQ][KSTEPS][2];
 #pragma unroll
     for (int nt = 0; nt < NQ; ++nt) {
-      const int part = QS == 2 ? (g & 1) : 0;
+      const bool lo_col = QS == 2 && (g & 1);
 #pragma unroll
       for (int j = 0; j < KSTEPS; ++j)
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int e = (2 * j + r) % (16 / C::BK);
-          __half hv[2];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const float v = ldexpf(qraw[nt][j][2 * r + h2], eq - field_pos<C::BK>(e));
-            const __half hi = __float2half_rn(v);
-            hv[h2] = part ? __float2half_rn(v - __half2float(hi)) : hi;
-          }
-          bq[nt][j][r] = pack_half2(hv[0], hv[1]);
+          const float f = pow2i(eq - field_pos<C::BK>(e));
+          const float v0 = qraw[nt][j][2 * r] * f, v1 = qraw[nt][j][2 * r + 1] * f;
+          const uint32_t hi = f2_to_h2(v0, v1);
+          const float2 h = unpack_half2(hi);
+          const uint32_t lo = f2_to_h2(v0 - h.x, v1 - h.y);
+          bq[nt][j][r] = lo_col ? lo : hi;
         }
     }
-    // sum of q over each group, in the same units as the code products:
-    // the score product of an all-ones code matrix.
-    float qsum[NG][NQ][4];
+    // Sum of q over each group, in the same units as the code products (the
+    // score product of an all-ones code matrix), times the softmax scale.
+    // qz[gr][nt] = {col 2c, col 2c+1}; for QS == 2 both columns of a lane
+    // belong to one head and are summed.
+    const float F = a.sm_scale_log2 * pow2i(24 - eq);
+    float2 qz[NG][NQ];
+    {
+      float qsum[NG][NQ][4];
 #pragma unroll
-    for (int gr = 0; gr < NG; ++gr)
+      for (int j = 0; j < KSTEPS; ++j) {
+        const int gr = 16 * j / G;
+        const uint32_t one0 = 0x00010001u << field_pos<C::BK>((2 * j) % (16 / C::BK));
+        const uint32_t one1 = 0x00010001u << field_pos<C::BK>((2 * j + 1) % (16 / C::BK));
 #pragma unroll
-      for (int nt = 0; nt < NQ; ++nt)
+        for (int nt = 0; nt < NQ; ++nt) {
+          if (j % (G / 16) == 0)
+            mma_f16_16816_zc(qsum[gr][nt], one0, one0, one1, one1, bq[nt][j][0], bq[nt][j][1]);
+          else
+            mma_f16_16816(qsum[gr][nt], one0, one0, one1, one1, bq[nt][j][0], bq[nt][j][1]);
+        }
+      }
 #pragma unroll
-        for (int r = 0; r < 4; ++r) qsum[gr][nt][r] = 0.0f;
+      for (int gr = 0; gr < NG; ++gr)
 #pragma unroll
-    for (int j = 0; j < KSTEPS; ++j) {
-      const int gr = 16 * j / G;
-      const uint32_t one0 = 0x00010001u << field_pos<C::BK>((2 * j) % (16 / C::BK));
-      const uint32_t one1 = 0x00010001u << field_pos<C::BK>((2 * j + 1) % (16 / C::BK));
-#pragma unroll
-      for (int nt = 0; nt < NQ; ++nt)
-        mma_f16_16816(qsum[gr][nt], one0, one0, one1, one1, bq[nt][j][0], bq[nt][j][1]);
+        for (int nt = 0; nt < NQ; ++nt)
+          qz[gr][nt] = QS == 2 ? make_float2((qsum[gr][nt][0] + qsum[gr][nt][1]) * F, 0.0f)
+                               : make_float2(qsum[gr][nt][0] * F, qsum[gr][nt][1] * F);
     }
-    const float F = ldexpf(a.sm_scale_log2, 24 - eq);
 
     // ------------------------------------------------------ main loop
-    float* wpex = pex + warp * 128;
+    // Softmax reference: m_run[hs] may lag the true running maximum by up to
+    // kLazy (log2 units), so weights p = 2^(logit - m_run) stay <= 2^kLazy;
+    // only a score above m_run + kLazy triggers the warp-wide maximum and
+    // the rescale of the accumulators.
+    constexpr float kLazy = 8.0f;
+    constexpr int TPW = C::TPW;
+    uint16_t* wb = wbuf + warp * TPW * C::WB_HALVES;
     float* walph = alph + warp * 8;
-    for (int it = 0; it < n_iters; ++it) {
-      const int s = it % C::kStages;
-      if (!mbar_wait_bounded(&full[s], (it / C::kStages) & 1, a.err)) break;
-      const int tb = t0 + it * C::kStageTokens + 16 * warp;
-      if (tb < t1) {
-        const int nvalid = t1 - tb;
-        const uint8_t* st = smem + s * C::STAGE_BYTES;
-        const uint8_t* kt = st + warp * 16 * C::KROW;
-        const uint8_t* vt = st + C::STAGE_K + warp * C::VTILE;
-        const uint32_t* kp =
-            reinterpret_cast<const uint32_t*>(st + C::STAGE_K + C::STAGE_V) + warp * 16 * NG;
-        const uint32_t* vp =
-            reinterpret_cast<const uint32_t*>(st + C::STAGE_K + C::STAGE_V + C::STAGE_P) +
-            warp * 16 * NG;
+    // lane offsets inside a stage (tile tt of this warp adds tt * 16 rows)
+    const int k_off = (warp * 16 * TPW + g) * C::KROW + c * C::KSLICE;
+    const int v_off = C::STAGE_K + warp * TPW * C::VTILE + lane * C::VP;
+    const int kp_off = C::STAGE_K + C::STAGE_V + (warp * 16 * TPW + g) * C::PROW;
+    uint32_t* const err = a.err;
+    const int n_tok = t1 - t0;
 
-        // ---- scores: S^T[token][head] = codes . q'
-        uint32_t kw[2 * C::KW];
-        lds_words<C::KSLICE>(kt + g * C::KROW + c * C::KSLICE, kw, 0);
-        lds_words<C::KSLICE>(kt + (g + 8) * C::KROW + c * C::KSLICE, kw, C::KW);
-        float acc[NG][NQ][4];
+    // Process NTL consecutive tiles of this warp (tile indices t_first ..),
+    // phase by phase so that their dependency chains interleave.  FULL:
+    // every position valid; otherwise a single tile with nvalid positions.
+    auto tiles_step = [&](auto full_tag, auto ntl_tag, const uint8_t* st, int t_first, int nvalid) {
+      constexpr bool FULL = decltype(full_tag)::value;
+      constexpr int NTL = decltype(ntl_tag)::value;
+      uint32_t kw[NTL][2 * C::KW];
+      uint32_t kpa[NTL][NG], kpb[NTL][NG], vpa[NTL][NG], vpb[NTL][NG];
 #pragma unroll
-        for (int gr = 0; gr < NG; ++gr)
+      for (int tt = 0; tt < NTL; ++tt) {
+        const int tix = t_first + tt;
+        lds_words<C::KSLICE>(st + k_off + tix * 16 * C::KROW, kw[tt], 0);
+        lds_words<C::KSLICE>(st + k_off + (tix * 16 + 8) * C::KROW, kw[tt], C::KW);
+        const uint32_t* kp = reinterpret_cast<const uint32_t*>(st + kp_off + tix * 16 * C::PROW);
+        const uint32_t* vq = reinterpret_cast<const uint32_t*>(st + kp_off + tix * 16 * C::PROW + C::STAGE_P);
 #pragma unroll
-          for (int nt = 0; nt < NQ; ++nt)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) acc[gr][nt][r] = 0.0f;
-#pragma unroll
-        for (int j = 0; j < KSTEPS; ++j) {
-          const int gr = 16 * j / G;
-          const uint32_t a0 = extract_codes<C::BK>(kw, 0, 2 * j);
-          const uint32_t a1 = extract_codes<C::BK>(kw, C::KW, 2 * j);
-          const uint32_t a2 = extract_codes<C::BK>(kw, 0, 2 * j + 1);
-          const uint32_t a3 = extract_codes<C::BK>(kw, C::KW, 2 * j + 1);
-#pragma unroll
-          for (int nt = 0; nt < NQ; ++nt)
-            mma_f16_16816(acc[gr][nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
+        for (int gr = 0; gr < NG; ++gr) {
+          kpa[tt][gr] = kp[gr];
+          kpb[tt][gr] = kp[8 * NG + gr];
+          vpa[tt][gr] = vq[gr];
+          vpb[tt][gr] = vq[8 * NG + gr];
         }
-        float sc[HT][2];
+      }
+      // ---- scores: S^T[token][col] = codes . q'
+      float acc[NTL][NG][NQ][4];
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int row = g + 8 * rr;
-          float ks[NG], kz[NG];
+      for (int j = 0; j < KSTEPS; ++j) {
+        const int gr = 16 * j / G;
 #pragma unroll
-          for (int gr = 0; gr < NG; ++gr) {
-            const float2 f = unpack_half2(kp[row * NG + gr]);
-            ks[gr] = f.x;
-            kz[gr] = f.y;
-          }
+        for (int tt = 0; tt < NTL; ++tt) {
+          const uint32_t a0 = extract_codes<C::BK>(kw[tt], 0, 2 * j);
+          const uint32_t a1 = extract_codes<C::BK>(kw[tt], C::KW, 2 * j);
+          const uint32_t a2 = extract_codes<C::BK>(kw[tt], 0, 2 * j + 1);
+          const uint32_t a3 = extract_codes<C::BK>(kw[tt], C::KW, 2 * j + 1);
 #pragma unroll
           for (int nt = 0; nt < NQ; ++nt) {
-            float v[2];
+            if (j % (G / 16) == 0)
+              mma_f16_16816_zc(acc[tt][gr][nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
+            else
+              mma_f16_16816(acc[tt][gr][nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
+          }
+        }
+      }
+      // logits (log2 units) lg[tt][hs][row]: F * sum_g (scale_g acc_g + zero_g qsum_g)
+      float lg[NTL][HT][2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              float t = 0.0f;
+      for (int tt = 0; tt < NTL; ++tt) {
+        if constexpr (QS == 2) {
 #pragma unroll
-              for (int gr = 0; gr < NG; ++gr)
-                t = fmaf(ks[gr], acc[gr][nt][2 * rr + e], fmaf(kz[gr], qsum[gr][nt][2 * rr + e], t));
-              v[e] = t;
+          for (int nt = 0; nt < NQ; ++nt) {
+            float2 t = make_float2(0.0f, 0.0f), z = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int gr = 0; gr < NG; ++gr) {
+              // rows (g, g+8): high + low columns
+              const float2 sum = __fadd2_rn(make_float2(acc[tt][gr][nt][0], acc[tt][gr][nt][2]),
+                                            make_float2(acc[tt][gr][nt][1], acc[tt][gr][nt][3]));
+              t = __ffma2_rn(scales_of(kpa[tt][gr], kpb[tt][gr]), sum, t);
+              z = __ffma2_rn(zeros_of(kpa[tt][gr], kpb[tt][gr]),
+                             make_float2(qz[gr][nt].x, qz[gr][nt].x), z);
             }
-            const bool ok = row < nvalid;
-            if (QS == 2) {
-              sc[nt][rr] = ok ? (v[0] + v[1]) * F : -INFINITY;
-            } else {
-              sc[2 * nt][rr] = ok ? v[0] * F : -INFINITY;
-              sc[2 * nt + 1][rr] = ok ? v[1] * F : -INFINITY;
+            const float2 l2 = __ffma2_rn(t, make_float2(F, F), z);
+            lg[tt][nt][0] = l2.x;
+            lg[tt][nt][1] = l2.y;
+          }
+        } else {
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+#pragma unroll
+            for (int nt = 0; nt < NQ; ++nt) {
+              float2 t = make_float2(0.0f, 0.0f), z = make_float2(0.0f, 0.0f);
+#pragma unroll
+              for (int gr = 0; gr < NG; ++gr) {
+                const float2 sz = unpack_half2(rr ? kpb[tt][gr] : kpa[tt][gr]);
+                t = __ffma2_rn(make_float2(sz.x, sz.x),
+                               make_float2(acc[tt][gr][nt][2 * rr], acc[tt][gr][nt][2 * rr + 1]), t);
+                z = __ffma2_rn(make_float2(sz.y, sz.y), qz[gr][nt], z);
+              }
+              const float2 l2 = __ffma2_rn(t, make_float2(F, F), z);
+              lg[tt][2 * nt][rr] = l2.x;
+              lg[tt][2 * nt + 1][rr] = l2.y;
             }
           }
         }
+      }
+      if (!FULL) {
+        // positions past the end: no score, and scale = zero = 0 for values
+#pragma unroll
+        for (int hs = 0; hs < HT; ++hs) {
+          if (g >= nvalid) lg[0][hs][0] = -INFINITY;
+          if (g + 8 >= nvalid) lg[0][hs][1] = -INFINITY;
+        }
+#pragma unroll
+        for (int gr = 0; gr < NG; ++gr) {
+          if (g >= nvalid) vpa[0][gr] = 0u;
+          if (g + 8 >= nvalid) vpb[0][gr] = 0u;
+        }
+      }
 
-        // ---- online softmax (exp2 domain)
-        bool changed = false;
+      // ---- lazy online softmax (exp2 domain)
+      float lmax[HT];
+#pragma unroll
+      for (int hs = 0; hs < HT; ++hs) {
+        lmax[hs] = fmaxf(lg[0][hs][0], lg[0][hs][1]);
+#pragma unroll
+        for (int tt = 1; tt < NTL; ++tt) lmax[hs] = fmaxf(lmax[hs], fmaxf(lg[tt][hs][0], lg[tt][hs][1]));
+      }
+      bool need = false;
+#pragma unroll
+      for (int hs = 0; hs < HT; ++hs) need |= lmax[hs] > m_run[hs] + kLazy;
+      const bool changed = __any_sync(0xffffffffu, need);
+      if (changed) {
 #pragma unroll
         for (int hs = 0; hs < HT; ++hs) {
           const int head = QS == 2 ? 4 * hs + c : 8 * (hs / 2) + 2 * c + (hs & 1);
-          const float mt = warp_max_xor(fmaxf(sc[hs][0], sc[hs][1]), 4);
+          const float mt = warp_max_xor(lmax[hs], 4);
           const float mnew = fmaxf(m_run[hs], mt);
-          changed |= mnew > m_run[hs];
-          const float alpha = mnew == -INFINITY ? 1.0f : exp2f(m_run[hs] - mnew);
-          const float mref = mnew == -INFINITY ? 0.0f : mnew;
-          const float p0 = exp2f(sc[hs][0] - mref);
-          const float p1 = exp2f(sc[hs][1] - mref);
-          l_run[hs] = fmaf(l_run[hs], alpha, p0 + p1);
+          const float alpha = mnew == -INFINITY ? 1.0f : exp2_approx(m_run[hs] - mnew);
+          l_run[hs] *= alpha;
+#pragma unroll
+          for (int gr = 0; gr < NG; ++gr)
+            zacc[hs][gr] = __fmul2_rn(zacc[hs][gr], make_float2(alpha, alpha));
           m_run[hs] = mnew;
-          wpex[g * 8 + head] = p0;
-          wpex[(g + 8) * 8 + head] = p1;
           if (g == 0) walph[head] = alpha;
         }
-        __syncwarp();
-        changed = __any_sync(0xffffffffu, changed);
-
-        // ---- weights p * scale_v as binary16 high/low parts (B operand).
-        // They are scaled by 2^u_run with u_run chosen from the largest value
-        // scale in the tile (p <= 1), so that the largest weight stays below
-        // 2^15 and the low part of every weight that matters stays a normal
-        // binary16.  When a tile needs a smaller exponent, the output
-        // accumulators are rescaled by the (exact) power of two.
-        const int kk[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
-        float2 svz[4][NG];
-        float smax = 0.0f;
+      }
+      float2 pr[NTL][HT];  // weights of rows (g, g+8)
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
+      for (int hs = 0; hs < HT; ++hs) {
+        const float mref = m_run[hs] == -INFINITY ? 0.0f : m_run[hs];
+#pragma unroll
+        for (int tt = 0; tt < NTL; ++tt) {
+          pr[tt][hs] = make_float2(exp2_approx(lg[tt][hs][0] - mref), exp2_approx(lg[tt][hs][1] - mref));
+          l_run[hs] += pr[tt][hs].x + pr[tt][hs].y;
+        }
+      }
+      // ---- exponent u of the output weights: keep p*scale*2^u < 2^15
+      {
+        uint32_t hm = vpa[0][0];
+#pragma unroll
+        for (int tt = 0; tt < NTL; ++tt)
 #pragma unroll
           for (int gr = 0; gr < NG; ++gr) {
-            svz[x][gr] = unpack_half2(vp[kk[x] * NG + gr]);
-            if (kk[x] < nvalid) smax = fmaxf(smax, svz[x][gr].x);
+            __half2 r = __hmax2(*reinterpret_cast<__half2*>(&hm), *reinterpret_cast<__half2*>(&vpa[tt][gr]));
+            r = __hmax2(r, *reinterpret_cast<__half2*>(&vpb[tt][gr]));
+            hm = *reinterpret_cast<uint32_t*>(&r);
           }
-        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 1));
-        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 2));
-        const int u_need = smax > 0.0f ? min(100, 14 - ilogbf(smax)) : 100;
-        const bool u_changed = u_need < u_run;
-        const float u_shift = u_changed ? __int_as_float((127 + u_need - u_run) << 23) : 1.0f;
-        if (u_changed) u_run = u_need;
-        const float f_u = __int_as_float((127 + u_run) << 23);
-        uint32_t bp[NP][NG][2];
+        float smax = unpack_half2(hm).x;
+        if (__any_sync(0xffffffffu, smax >= u_bound)) {
+          smax = warp_max_xor(smax, 4);
+          const int u_need = min(u_run, 6 - ilogbf(smax));
+          const float shift = pow2i(u_need - u_run);
+          u_run = u_need;
+          u_bound = pow2i(7 - u_run);
+#pragma unroll
+          for (int j = 0; j < KSTEPS; ++j)
+#pragma unroll
+            for (int pt = 0; pt < NP; ++pt)
+#pragma unroll
+              for (int r = 0; r < 4; ++r) oacc[j][pt][r] *= shift;
+        }
+      }
+      // ---- weights p * scale_v * 2^u of rows (g, g+8), binary16 high and
+      // low parts, staged so that each B-fragment register is one load;
+      // zero term accumulated here.
+      {
+        const float fu = pow2i(u_run);
+#pragma unroll
+        for (int tt = 0; tt < NTL; ++tt) {
+          uint16_t* wbt = wb + (t_first + tt) * C::WB_HALVES;
+#pragma unroll
+          for (int gr = 0; gr < NG; ++gr) {
+            const float2 sc = scales_of(vpa[tt][gr], vpb[tt][gr]);
+            const float2 zr = zeros_of(vpa[tt][gr], vpb[tt][gr]);
+#pragma unroll
+            for (int hs = 0; hs < HT; ++hs) {
+              const int head = QS == 2 ? 4 * hs + c : 8 * (hs / 2) + 2 * c + (hs & 1);
+              const float2 P = __fmul2_rn(__fmul2_rn(pr[tt][hs], make_float2(fu, fu)), sc);
+              const uint32_t hi = f2_to_h2(P.x, P.y);
+              const float2 hf = unpack_half2(hi);
+              const uint32_t lo = f2_to_h2(P.x - hf.x, P.y - hf.y);
+              uint16_t* row = wbt + (gr * 8 + head) * 2 * C::WB_RS;
+              row[g] = static_cast<uint16_t>(hi);
+              row[g + 8] = static_cast<uint16_t>(hi >> 16);
+              row[C::WB_RS + g] = static_cast<uint16_t>(lo);
+              row[C::WB_RS + g + 8] = static_cast<uint16_t>(lo >> 16);
+              zacc[hs][gr] = __ffma2_rn(pr[tt][hs], zr, zacc[hs][gr]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (changed) {
 #pragma unroll
         for (int pt = 0; pt < NP; ++pt) {
-          const int hd = 4 * pt + (g >> 1);
-          const int part = g & 1;
-          float pv[4];
+          const float ao = walph[4 * pt + c];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) pv[x] = wpex[kk[x] * 8 + hd];
-          const float az = changed ? walph[hd] : 1.0f;
+          for (int j = 0; j < KSTEPS; ++j)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) oacc[j][pt][r] *= ao;
+        }
+      }
+      // ---- output: O^T[dim][col] += codes^T . (p * scale_v)
+      uint32_t bp[NTL][NP][NG][2];
+      uint32_t vw[NTL][C::VW];
+#pragma unroll
+      for (int tt = 0; tt < NTL; ++tt) {
+        const uint16_t* rd = wb + (t_first + tt) * C::WB_HALVES + g * C::WB_RS + 2 * c;
+#pragma unroll
+        for (int pt = 0; pt < NP; ++pt)
 #pragma unroll
           for (int gr = 0; gr < NG; ++gr) {
-            __half hv[4];
-            float z = 0.0f;
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              const float P = pv[x] == 0.0f ? 0.0f : (pv[x] * f_u) * svz[x][gr].x;
-              const __half hi = __float2half_rn(P);
-              hv[x] = part ? __float2half_rn(P - __half2float(hi)) : hi;
-              z += pv[x] == 0.0f ? 0.0f : pv[x] * svz[x][gr].y;
-            }
-            bp[pt][gr][0] = pack_half2(hv[0], hv[1]);
-            bp[pt][gr][1] = pack_half2(hv[2], hv[3]);
-            if (part == 0) zacc[pt][gr] = fmaf(zacc[pt][gr], az, z);
+            const uint16_t* row = rd + (gr * 8 + 4 * pt) * 2 * C::WB_RS;
+            bp[tt][pt][gr][0] = *reinterpret_cast<const uint32_t*>(row);
+            bp[tt][pt][gr][1] = *reinterpret_cast<const uint32_t*>(row + 8);
           }
-        }
-        if (changed || u_changed) {
-#pragma unroll
-          for (int pt = 0; pt < NP; ++pt) {
-            const float ao = (changed ? walph[4 * pt + c] : 1.0f) * u_shift;
-#pragma unroll
-            for (int j = 0; j < KSTEPS; ++j)
-#pragma unroll
-              for (int r = 0; r < 4; ++r) oacc[j][pt][r] *= ao;
-          }
-        }
-
-        // ---- output: O^T[dim][head] += codes^T . (p * scale_v)
-        uint32_t vw[C::VW];
 #pragma unroll
         for (int pc = 0; pc < C::VN / C::VP; ++pc)
-          lds_words<C::VP>(vt + pc * 32 * C::VP + lane * C::VP, vw, pc * (C::VP / 4));
+          lds_words<C::VP>(st + v_off + (t_first + tt) * C::VTILE + pc * 32 * C::VP, vw[tt],
+                           pc * (C::VP / 4));
+      }
 #pragma unroll
-        for (int j = 0; j < KSTEPS; ++j) {
-          const int gr = 16 * j / G;
-          const uint32_t a0 = extract_codes<C::BV>(vw, 0, 2 * j);
-          const uint32_t a1 = extract_codes<C::BV>(vw, 0, 2 * j + 1);
-          const uint32_t a2 = extract_codes<C::BV>(vw, C::WV, 2 * j);
-          const uint32_t a3 = extract_codes<C::BV>(vw, C::WV, 2 * j + 1);
+      for (int j = 0; j < KSTEPS; ++j) {
+        const int gr = 16 * j / G;
+#pragma unroll
+        for (int tt = 0; tt < NTL; ++tt) {
+          const uint32_t a0 = extract_codes<C::BV>(vw[tt], 0, 2 * j);
+          const uint32_t a1 = extract_codes<C::BV>(vw[tt], 0, 2 * j + 1);
+          const uint32_t a2 = extract_codes<C::BV>(vw[tt], C::WV, 2 * j);
+          const uint32_t a3 = extract_codes<C::BV>(vw[tt], C::WV, 2 * j + 1);
 #pragma unroll
           for (int pt = 0; pt < NP; ++pt)
-            mma_f16_16816(oacc[j][pt], a0, a1, a2, a3, bp[pt][gr][0], bp[pt][gr][1]);
+            mma_f16_16816(oacc[j][pt], a0, a1, a2, a3, bp[tt][pt][gr][0], bp[tt][pt][gr][1]);
         }
-        __syncwarp();
+      }
+      __syncwarp();
+    };
+
+    int s = 0;
+    uint32_t phase = 0;
+    for (int it = 0; it < n_iters; ++it) {
+      if (!mbar_wait_bounded(&full[s], phase, err)) break;
+      const uint8_t* st = smem + s * C::STAGE_BYTES;
+      const int base = it * C::kStageTokens + warp * 16 * TPW;  // first position of this warp
+      if (base + 16 * TPW <= n_tok) {
+        tiles_step(std::true_type{}, std::integral_constant<int, TPW>{}, st, 0, 16);
+      } else {
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt) {
+          const int rem = n_tok - (base + 16 * tt);
+          if (rem >= 16)
+            tiles_step(std::true_type{}, std::integral_constant<int, 1>{}, st, tt, 16);
+          else if (rem > 0)
+            tiles_step(std::false_type{}, std::integral_constant<int, 1>{}, st, tt, rem);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == C::kStages) {
+        s = 0;
+        phase ^= 1u;
+      }
     }
   }
 
   // ------------------------------------------------------------ epilogue
   __syncthreads();  // all stages consumed; the ring becomes the merge buffer
   float* ob = reinterpret_cast<float*>(smem);  // [warp][8][D]
-  float* mb = pex;                             // [warp][8]
-  float* lb = pex + 32;                        // [warp][8]
-  float* zb = pex + 64;                        // [warp][8][NG]
+  float* mb = mrg;                             // [warp][8]
+  float* lb = mb + C::kWarps * 8;              // [warp][8]
+  float* zb = lb + C::kWarps * 8;              // [warp][8][NG]
+  float* wt = zb + C::kWarps * 8 * NG;         // [head][warp] merge weights
+  float* rden = wt + 8 * C::kWarps;            // [head] 1 / denominator
   if (warp < C::kWarps) {
 #pragma unroll
     for (int hs = 0; hs < HT; ++hs) {
+      const int head = QS == 2 ? 4 * hs + c : 8 * (hs / 2) + 2 * c + (hs & 1);
       float l = l_run[hs];
       l += __shfl_xor_sync(0xffffffffu, l, 4);
       l += __shfl_xor_sync(0xffffffffu, l, 8);
       l += __shfl_xor_sync(0xffffffffu, l, 16);
-      const int head = QS == 2 ? 4 * hs + c : 8 * (hs / 2) + 2 * c + (hs & 1);
+      float z[NG];
+#pragma unroll
+      for (int gr = 0; gr < NG; ++gr) {
+        z[gr] = zacc[hs][gr].x + zacc[hs][gr].y;
+        z[gr] += __shfl_xor_sync(0xffffffffu, z[gr], 4);
+        z[gr] += __shfl_xor_sync(0xffffffffu, z[gr], 8);
+        z[gr] += __shfl_xor_sync(0xffffffffu, z[gr], 16);
+      }
       if (g == 0) {
         mb[warp * 8 + head] = m_run[hs];
         lb[warp * 8 + head] = l;
+#pragma unroll
+        for (int gr = 0; gr < NG; ++gr) zb[(warp * 8 + head) * NG + gr] = z[gr];
       }
     }
-#pragma unroll
-    for (int pt = 0; pt < NP; ++pt)
-#pragma unroll
-      for (int gr = 0; gr < NG; ++gr) {
-        float z = zacc[pt][gr];
-        z += __shfl_xor_sync(0xffffffffu, z, 1);
-        z += __shfl_xor_sync(0xffffffffu, z, 2);
-        if ((g & 1) == 0 && c == 0) zb[(warp * 8 + 4 * pt + (g >> 1)) * NG + gr] = z;
-      }
 #pragma unroll
     for (int pt = 0; pt < NP; ++pt) {
       const int head = 4 * pt + c;
 #pragma unroll
       for (int j = 0; j < KSTEPS; ++j) {
-        const float s0 = ldexpf(1.0f, 24 - u_run - field_pos<C::BV>((2 * j) % (16 / C::BV)));
-        const float s1 = ldexpf(1.0f, 24 - u_run - field_pos<C::BV>((2 * j + 1) % (16 / C::BV)));
+        const float s0 = pow2i(24 - u_run - field_pos<C::BV>((2 * j) % (16 / C::BV)));
+        const float s1 = pow2i(24 - u_run - field_pos<C::BV>((2 * j + 1) % (16 / C::BV)));
         ob[(warp * 8 + head) * D + 16 * j + g] = (oacc[j][pt][0] + oacc[j][pt][1]) * s0;
         ob[(warp * 8 + head) * D + 16 * j + 8 + g] = (oacc[j][pt][2] + oacc[j][pt][3]) * s1;
       }
     }
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < nh * D; idx += C::kThreads) {
-    const int head = idx / D, d = idx % D;
+  if (threadIdx.x < nh) {
+    const int head = threadIdx.x;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < C::kWarps; ++w) M = fmaxf(M, mb[w * 8 + head]);
-    float num = 0.0f, den = 0.0f;
+    float den = 0.0f;
 #pragma unroll
     for (int w = 0; w < C::kWarps; ++w) {
       const float mw = mb[w * 8 + head];
-      if (mw == -INFINITY) continue;
-      const float wt = exp2f(mw - M);
-      num = fmaf(wt, ob[(w * 8 + head) * D + d] + zb[(w * 8 + head) * NG + d / G], num);
-      den = fmaf(wt, lb[w * 8 + head], den);
+      const float x = mw == -INFINITY ? 0.0f : exp2_approx(mw - M);
+      wt[head * C::kWarps + w] = x;
+      den = fmaf(x, lb[w * 8 + head], den);
     }
+    rden[head] = __frcp_rn(den);
     const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * a.num_splits + split;
-    a.ws_o[row * D + d] = num / den;
-    if (d == 0) a.ws_lse[row] = M + log2f(den);
+    a.ws_lse[row] = M + __log2f(den);
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < nh * D; idx += C::kThreads) {
+    const int head = idx / D, d = idx % D;
+    float num = 0.0f;
+#pragma unroll
+    for (int w = 0; w < C::kWarps; ++w)
+      num = fmaf(wt[head * C::kWarps + w], ob[(w * 8 + head) * D + d] + zb[(w * 8 + head) * NG + d / G], num);
+    const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * a.num_splits + split;
+    a.ws_o[row * D + d] = num * rden[head];
   }
 }
 
@@ -518,12 +703,14 @@ DecodeKernel make_decode_kernel() {
 }
 
 // Instances for one (bits_k, bits_v) pair: D in {64, 128}, groups per row,
-// and the four query variants.
+// and the query variants: up to 4 heads per CTA (any query type: one head per
+// lane, high/low columns), 5..8 heads with 16-bit queries (two heads per
+// lane), 5..8 heads with binary32 queries (high/low columns, two n-tiles).
 template <int BK, int BV>
 bool get_decode_kernel_bits(int head_dim, int num_groups, int variant, DecodeKernel* out) {
 #define KVQ_VARIANTS(D, NG)                                                        \
   switch (variant) {                                                               \
-    case 0: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NG, 1, 1, 1>>(); return true; \
+    case 0:                                                                        \
     case 1: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NG, 2, 1, 1>>(); return true; \
     case 2: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NG, 1, 1, 2>>(); return true; \
     case 3: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NG, 2, 2, 2>>(); return true; \
