@@ -117,13 +117,12 @@ int variant_of(int heads_per_cta, int q_dtype) {
   return (heads_per_cta <= 4 ? 0 : 2) + (q_dtype == KVQ_F32 ? 1 : 0);
 }
 
-// Split-K plan.  Tokens per split are a multiple of the 64-token stage.
-// When one wave of resident CTAs can cover every (batch row, kv head) with
-// splits of at least 256 tokens, use exactly one wave (equal lengths finish
-// together, nothing waits for a second wave).  Otherwise aim at about four
-// waves, so that the block scheduler can balance ragged lengths, with at
-// least 256 tokens per split (partial-result traffic).  The plan depends
-// only on the shape, Hq, max_seq_len and the device.
+// Split-K plan.  Tokens per split are a multiple of 64.  Aim at about four
+// waves of resident CTAs, so that the block scheduler can balance ragged
+// lengths; when that would cut splits below 1024 tokens (small problems),
+// aim at one wave instead, with at least 256 tokens per split (per-CTA
+// set-up and partial-result traffic).  The plan depends only on the shape,
+// Hq, max_seq_len and the device.
 int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
   const int gq = Hq / c->kv_heads;
   p->heads_per_cta = gq < 8 ? gq : 8;
@@ -151,15 +150,9 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
   const long long units = static_cast<long long>(c->batch) * c->kv_heads * p->head_groups;
   const long long slots = static_cast<long long>(sms) * per_sm;
   const long long max64 = (max_seq_len + 63LL) / 64 * 64;
-  long long split = 0;
-  if (units <= slots) {
-    const long long per_unit = slots / units;
-    split = ((max_seq_len + per_unit - 1) / per_unit + 63) / 64 * 64;
-  }
-  if (split < 256) {
-    const long long want = 4 * slots;
-    split = ((units * max_seq_len + want - 1) / want + 63) / 64 * 64;
-  }
+  const long long work = units * max_seq_len;
+  long long split = ((work + 4 * slots - 1) / (4 * slots) + 63) / 64 * 64;
+  if (split < 1024) split = ((work + slots - 1) / slots + 63) / 64 * 64;
   if (split < 256) split = 256;
   if (split > max64) split = max64;
   if (const char* env = std::getenv("KVQ_SPLIT_TOKENS")) {

@@ -37,8 +37,8 @@ namespace kvq {
 template <int D_, int BK_, int BV_, int NG_, int QS_, int NQ_, int NP_>
 struct DecodeCfg {
   static constexpr int D = D_, BK = BK_, BV = BV_, NG = NG_, QS = QS_, NQ = NQ_, NP = NP_;
-  static constexpr int kWarps = 4;  // consumer warps
-  static constexpr int kThreads = 32 * (kWarps + 1);
+  static constexpr int kWarps = 4;  // warps per CTA; each runs its own copy pipeline
+  static constexpr int kThreads = 32 * kWarps;
   static constexpr int TPW = 2;     // 16-token tiles per warp per stage
   static constexpr int kStageTokens = 16 * TPW * kWarps;
   static constexpr int G = D / NG;
@@ -52,23 +52,24 @@ struct DecodeCfg {
   static constexpr int VW = VN / 4;
   static constexpr int WV = D * BV / 128;  // V words per half-lane
   static constexpr int PROW = NG * 4;
-  static constexpr int STAGE_K = kStageTokens * KROW;
-  static constexpr int STAGE_V = TPW * kWarps * VTILE;
-  static constexpr int STAGE_P = kStageTokens * PROW;
-  static constexpr int STAGE_BYTES = STAGE_K + STAGE_V + 2 * STAGE_P;
-  static constexpr int kStages = STAGE_BYTES > 20000 ? 3 : 4;
-  static constexpr int RING_BYTES = kStages * STAGE_BYTES;
-  // staged output weights: per warp [group][head][part][WB_RS halves]
+  // one slot = one warp's 16*TPW positions of a stage: K rows, V tiles, K params, V params
+  static constexpr int SLOT_K = 16 * TPW * KROW;
+  static constexpr int SLOT_V = TPW * VTILE;
+  static constexpr int SLOT_P = 16 * TPW * PROW;
+  static constexpr int SLOT_BYTES = SLOT_K + SLOT_V + 2 * SLOT_P;
+  static constexpr int kSlots = SLOT_BYTES > 6144 ? 2 : 3;  // copies in flight per warp
+  static constexpr int RING_BYTES = kWarps * kSlots * SLOT_BYTES;
+  // staged output weights: per warp and tile [group][head][part][WB_RS halves]
   static constexpr int WB_RS = 24;  // halves per row: 16 positions + pad (conflict-free)
   static constexpr int WB_HALVES = NG * 8 * 2 * WB_RS;
   static constexpr int WB_BYTES = TPW * kWarps * WB_HALVES * 2;
   static constexpr int ALPHA_FLOATS = kWarps * 8;
   static constexpr int MERGE_FLOATS = kWarps * 8 * (2 + NG) + 2 * 8 * (kWarps + 1);
   static constexpr int SMEM_BYTES =
-      RING_BYTES + WB_BYTES + 4 * (ALPHA_FLOATS + MERGE_FLOATS) + 16 * kStages;
+      RING_BYTES + WB_BYTES + 4 * (ALPHA_FLOATS + MERGE_FLOATS) + 8 * kWarps * kSlots;
   static constexpr int HT = QS == 1 ? 2 * NQ : NQ;  // score head slots per lane
   static_assert(RING_BYTES >= kWarps * 8 * D * 4, "merge buffer must fit in the ring");
-  static_assert(STAGE_BYTES % 16 == 0 && STAGE_K % 16 == 0 && STAGE_V % 16 == 0, "alignment");
+  static_assert(SLOT_BYTES % 16 == 0 && SLOT_K % 16 == 0 && SLOT_V % 16 == 0, "alignment");
   static_assert(G >= 16 && G % 16 == 0, "group must cover whole 16-element steps");
 };
 
@@ -162,8 +163,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   uint16_t* wbuf = reinterpret_cast<uint16_t*>(smem + C::RING_BYTES);  // staged weights
   float* alph = reinterpret_cast<float*>(smem + C::RING_BYTES + C::WB_BYTES);  // [warp][8]
   float* mrg = alph + C::ALPHA_FLOATS;                                     // merge area
-  uint64_t* full = reinterpret_cast<uint64_t*>(mrg + C::MERGE_FLOATS);
-  uint64_t* empty = full + C::kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(mrg + C::MERGE_FLOATS);    // [warp][slot]
 
   const int split = blockIdx.x;
   const int hk = blockIdx.y / a.head_groups;
@@ -181,53 +181,41 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   const int t0 = split * a.split_tokens;
   if (t0 >= len) return;
   const int t1 = min(t0 + a.split_tokens, len);
-  const int n_iters = (t1 - t0 + C::kStageTokens - 1) / C::kStageTokens;
+  const int n_tok = t1 - t0;
   const int head0 = hk * a.gq + hg * a.heads_per_cta;
   const int nh = min(a.heads_per_cta, a.gq - hg * a.heads_per_cta);
   const size_t slot = static_cast<size_t>(b) * a.kv_heads + hk;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C::kWarps);
-    }
+  // ---- this warp's copy pipeline: positions [it*kStageTokens + 16*TPW*warp, +16*TPW)
+  // of the split for it = 0 .. my_iters-1, kSlots copies in flight.
+  const int my_first = warp * 16 * C::TPW;
+  const int my_iters = n_tok > my_first ? (n_tok - my_first + C::kStageTokens - 1) / C::kStageTokens : 0;
+  uint64_t* wfull = full + warp * C::kSlots;
+  uint8_t* wring = smem + warp * C::kSlots * C::SLOT_BYTES;
+  const uint8_t* kb = a.k_codes + slot * a.capacity * C::KROW;
+  const uint8_t* vb = a.v_codes + slot * (a.capacity / 16) * C::VTILE;
+  const uint8_t* kpb = reinterpret_cast<const uint8_t*>(a.k_params) + slot * a.capacity * C::PROW;
+  const uint8_t* vpb = reinterpret_cast<const uint8_t*>(a.v_params) + slot * a.capacity * C::PROW;
+  auto issue = [&](int it, int sl) {
+    const int base = it * C::kStageTokens + my_first;  // multiple of 16
+    const int n16 = (min(16 * C::TPW, n_tok - base) + 15) & ~15;
+    const int tb = t0 + base;
+    uint8_t* dst = wring + sl * C::SLOT_BYTES;
+    const uint32_t kbytes = n16 * C::KROW, vbytes = (n16 / 16) * C::VTILE, pbytes = n16 * C::PROW;
+    mbar_arrive_expect_tx(&wfull[sl], kbytes + vbytes + 2 * pbytes);
+    bulk_copy_g2s(dst, kb + static_cast<size_t>(tb) * C::KROW, kbytes, &wfull[sl]);
+    bulk_copy_g2s(dst + C::SLOT_K, vb + static_cast<size_t>(tb / 16) * C::VTILE, vbytes, &wfull[sl]);
+    bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V, kpb + static_cast<size_t>(tb) * C::PROW, pbytes,
+                  &wfull[sl]);
+    bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V + C::SLOT_P, vpb + static_cast<size_t>(tb) * C::PROW,
+                  pbytes, &wfull[sl]);
+  };
+  if (lane == 0) {
+    for (int sl = 0; sl < C::kSlots; ++sl) mbar_init(&wfull[sl], 1);
     fence_barrier_init();
+    for (int it = 0; it < min(C::kSlots, my_iters); ++it) issue(it, it);
   }
-  __syncthreads();
-
-  if (warp == C::kWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint8_t* kb = a.k_codes + slot * a.capacity * C::KROW;
-      const uint8_t* vb = a.v_codes + slot * (a.capacity / 16) * C::VTILE;
-      const uint8_t* kpb = reinterpret_cast<const uint8_t*>(a.k_params) + slot * a.capacity * C::PROW;
-      const uint8_t* vpb = reinterpret_cast<const uint8_t*>(a.v_params) + slot * a.capacity * C::PROW;
-      int issued = 0;
-      for (int it = 0; it < n_iters; ++it) {
-        const int s = it % C::kStages;
-        if (it >= C::kStages && !mbar_wait_bounded(&empty[s], ((it / C::kStages) + 1) & 1, a.err))
-          break;
-        const int tb = t0 + it * C::kStageTokens;
-        const int n16 = (min(C::kStageTokens, t1 - tb) + 15) & ~15;
-        uint8_t* st = smem + s * C::STAGE_BYTES;
-        const uint32_t kbytes = n16 * C::KROW, vbytes = (n16 / 16) * C::VTILE,
-                       pbytes = n16 * C::PROW;
-        mbar_arrive_expect_tx(&full[s], kbytes + vbytes + 2 * pbytes);
-        bulk_copy_g2s(st, kb + static_cast<size_t>(tb) * C::KROW, kbytes, &full[s]);
-        bulk_copy_g2s(st + C::STAGE_K, vb + static_cast<size_t>(tb / 16) * C::VTILE, vbytes,
-                      &full[s]);
-        bulk_copy_g2s(st + C::STAGE_K + C::STAGE_V, kpb + static_cast<size_t>(tb) * C::PROW,
-                      pbytes, &full[s]);
-        bulk_copy_g2s(st + C::STAGE_K + C::STAGE_V + C::STAGE_P,
-                      vpb + static_cast<size_t>(tb) * C::PROW, pbytes, &full[s]);
-        ++issued;
-      }
-      // Drain: every copy issued must have landed before shared memory is
-      // reused below (normally already true; bounded in any case).
-      for (int it = max(0, issued - C::kStages); it < issued; ++it)
-        mbar_wait_bounded(&full[it % C::kStages], (it / C::kStages) & 1, a.err);
-    }
-  }
+  __syncwarp();
 
   // ------------------------------------------------------------ consumers
   const int g = lane >> 2, c = lane & 3;
@@ -254,7 +242,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
 #pragma unroll
     for (int gr = 0; gr < NG; ++gr) zacc[hs][gr] = make_float2(0.0f, 0.0f);
 
-  if (warp < C::kWarps) {
+  {
     // -------- query fragments (B operand of the score product), once per CTA
     float qraw[NQ][KSTEPS][4];
     float amax = 0.0f;
@@ -343,11 +331,10 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     uint16_t* wb = wbuf + warp * TPW * C::WB_HALVES;
     float* walph = alph + warp * 8;
     // lane offsets inside a stage (tile tt of this warp adds tt * 16 rows)
-    const int k_off = (warp * 16 * TPW + g) * C::KROW + c * C::KSLICE;
-    const int v_off = C::STAGE_K + warp * TPW * C::VTILE + lane * C::VP;
-    const int kp_off = C::STAGE_K + C::STAGE_V + (warp * 16 * TPW + g) * C::PROW;
+    const int k_off = g * C::KROW + c * C::KSLICE;
+    const int v_off = C::SLOT_K + lane * C::VP;
+    const int kp_off = C::SLOT_K + C::SLOT_V + g * C::PROW;
     uint32_t* const err = a.err;
-    const int n_tok = t1 - t0;
 
     // Process NTL consecutive tiles of this warp (tile indices t_first ..),
     // phase by phase so that their dependency chains interleave.  FULL:
@@ -363,7 +350,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         lds_words<C::KSLICE>(st + k_off + tix * 16 * C::KROW, kw[tt], 0);
         lds_words<C::KSLICE>(st + k_off + (tix * 16 + 8) * C::KROW, kw[tt], C::KW);
         const uint32_t* kp = reinterpret_cast<const uint32_t*>(st + kp_off + tix * 16 * C::PROW);
-        const uint32_t* vq = reinterpret_cast<const uint32_t*>(st + kp_off + tix * 16 * C::PROW + C::STAGE_P);
+        const uint32_t* vq = reinterpret_cast<const uint32_t*>(st + kp_off + tix * 16 * C::PROW + C::SLOT_P);
 #pragma unroll
         for (int gr = 0; gr < NG; ++gr) {
           kpa[tt][gr] = kp[gr];
@@ -586,12 +573,13 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       __syncwarp();
     };
 
-    int s = 0;
+    int sl = 0;
     uint32_t phase = 0;
-    for (int it = 0; it < n_iters; ++it) {
-      if (!mbar_wait_bounded(&full[s], phase, err)) break;
-      const uint8_t* st = smem + s * C::STAGE_BYTES;
-      const int base = it * C::kStageTokens + warp * 16 * TPW;  // first position of this warp
+    int it = 0;
+    for (; it < my_iters; ++it) {
+      if (!mbar_wait_bounded(&wfull[sl], phase, err)) break;
+      const uint8_t* st = wring + sl * C::SLOT_BYTES;
+      const int base = it * C::kStageTokens + my_first;  // first position of this slot
       if (base + 16 * TPW <= n_tok) {
         tiles_step(std::true_type{}, std::integral_constant<int, TPW>{}, st, 0, 16);
       } else {
@@ -605,11 +593,22 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      if (++s == C::kStages) {
-        s = 0;
+      if (lane == 0 && it + C::kSlots < my_iters) {
+        // the warp's reads of this slot are done (registers); hand it back to
+        // the copy engine for a later stage
+        fence_proxy_async_shared();
+        issue(it + C::kSlots, sl);
+      }
+      if (++sl == C::kSlots) {
+        sl = 0;
         phase ^= 1u;
       }
+    }
+    // Drain (only after a timed-out wait): copies issued but not consumed
+    // must land before shared memory is reused; bounded in any case.
+    if (it < my_iters && lane == 0) {
+      for (int k = it; k < min(my_iters, it + C::kSlots); ++k)
+        mbar_wait_bounded(&wfull[k % C::kSlots], (k / C::kSlots) & 1, err);
     }
   }
 
@@ -621,7 +620,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   float* zb = lb + C::kWarps * 8;              // [warp][8][NG]
   float* wt = zb + C::kWarps * 8 * NG;         // [head][warp] merge weights
   float* rden = wt + 8 * C::kWarps;            // [head] 1 / denominator
-  if (warp < C::kWarps) {
+  {
 #pragma unroll
     for (int hs = 0; hs < HT; ++hs) {
       const int head = QS == 2 ? 4 * hs + c : 8 * (hs / 2) + 2 * c + (hs & 1);
