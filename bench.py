@@ -76,7 +76,7 @@ def sha_of(paths):
 
 
 KERNEL_SOURCES = {
-    "quantize": ["kv_cache_mixed_kvq_b200/csrc/quantize.cu", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
+    "quantize": ["kv_cache_mixed_kvq_b200/csrc/quantize.cuh", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
     "decode": ["kv_cache_mixed_kvq_b200/csrc/decode.cuh", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
 }
 
@@ -103,6 +103,15 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except (OSError, ValueError, KeyError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank float over all ranks (one all-reduce; identity at N=1)."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ----------------------------------------------------------------- clocks
@@ -257,11 +266,7 @@ def run_ours(args, rank, world, device):
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, device)
     ms_step = ms / args.steps
     flags = arm.kvq.kvq_device_error_flags()
 
@@ -394,11 +399,7 @@ def run_e2e(arm, args, step_bytes, world, device):
         one()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, device)
     h2d = (hk.numel() * hk.element_size() + hv.numel() * hv.element_size() +
            hq.numel() * hq.element_size()) if arm.n_new else hq.numel() * hq.element_size()
     return {"value": round(world * step_bytes / (ms / 1e3) / 1e9, 2), "unit": "GB/s",

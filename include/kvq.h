@@ -275,6 +275,13 @@ int32_t kvq_decode_split_tokens(const kvq_cache_desc* cache,
  */
 int kvq_device_error_flags(kvq_stream_t stream, uint32_t* flags);
 
+/*
+ * The same read-and-clear in one return value: the error word's bits
+ * (kvq_device_error, >= 0) after synchronizing `stream`, or -KVQ_ERR_CUDA
+ * if the copy or the synchronization failed.
+ */
+int kvq_last_device_error(kvq_stream_t stream);
+
 /* Static text for a kvq_status value. */
 const char* kvq_strerror(int32_t status);
 

@@ -78,6 +78,8 @@ def library() -> ctypes.CDLL:
     lib.kvq_decode_attention.restype = ctypes.c_int
     lib.kvq_device_error_flags.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
     lib.kvq_device_error_flags.restype = ctypes.c_int
+    lib.kvq_last_device_error.argtypes = [P]
+    lib.kvq_last_device_error.restype = ctypes.c_int
     lib.kvq_strerror.argtypes = [I32]
     lib.kvq_strerror.restype = ctypes.c_char_p
     _lib = lib
@@ -206,3 +208,11 @@ def kvq_device_error_flags(stream: Optional[torch.cuda.Stream] = None) -> int:
     st = library().kvq_device_error_flags(_stream_ptr(stream), ctypes.byref(flags))
     _check(st, "kvq_device_error_flags")
     return int(flags.value)
+
+
+def kvq_last_device_error(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Error-word bits (read and cleared); raises KvqError on a CUDA failure."""
+    r = library().kvq_last_device_error(_stream_ptr(stream))
+    if r < 0:
+        _check(-r, "kvq_last_device_error")
+    return int(r)

@@ -117,12 +117,13 @@ int variant_of(int heads_per_cta, int q_dtype) {
   return (heads_per_cta <= 4 ? 0 : 2) + (q_dtype == KVQ_F32 ? 1 : 0);
 }
 
-// Split-K plan.  Tokens per split are a multiple of 64.  Aim at about four
-// waves of resident CTAs, so that the block scheduler can balance ragged
-// lengths; when that would cut splits below 1024 tokens (small problems),
-// aim at one wave instead, with at least 256 tokens per split (per-CTA
-// set-up and partial-result traffic).  The plan depends only on the shape,
-// Hq, max_seq_len and the device.
+// Split-K plan.  Tokens per split are a multiple of 64, at least 256 (per-CTA
+// set-up and partial-result traffic).  When one wave of resident CTAs gives
+// every (batch row, kv head, head group) at least four splits, use exactly one
+// wave: splits are rounded up, so the grid never spills into a second wave.
+// Otherwise aim at about four waves, so that the block scheduler can balance
+// ragged lengths.  The plan depends only on the shape, Hq, max_seq_len and
+// the device.
 int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
   const int gq = Hq / c->kv_heads;
   p->heads_per_cta = gq < 8 ? gq : 8;
@@ -150,9 +151,14 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
   const long long units = static_cast<long long>(c->batch) * c->kv_heads * p->head_groups;
   const long long slots = static_cast<long long>(sms) * per_sm;
   const long long max64 = (max_seq_len + 63LL) / 64 * 64;
-  const long long work = units * max_seq_len;
-  long long split = ((work + 4 * slots - 1) / (4 * slots) + 63) / 64 * 64;
-  if (split < 1024) split = ((work + slots - 1) / slots + 63) / 64 * 64;
+  const long long per_unit = slots / units;
+  long long split;
+  if (per_unit >= 4) {
+    split = ((max_seq_len + per_unit - 1) / per_unit + 63) / 64 * 64;
+  } else {
+    const long long work = units * max_seq_len;
+    split = ((work + 4 * slots - 1) / (4 * slots) + 63) / 64 * 64;
+  }
   if (split < 256) split = 256;
   if (split > max64) split = max64;
   if (const char* env = std::getenv("KVQ_SPLIT_TOKENS")) {
@@ -351,6 +357,12 @@ int kvq_device_error_flags(kvq_stream_t stream, uint32_t* flags) {
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
   *flags = host;
   return KVQ_OK;
+}
+
+int kvq_last_device_error(kvq_stream_t stream) {
+  uint32_t flags = 0;
+  const int st = kvq_device_error_flags(stream, &flags);
+  return st == KVQ_OK ? static_cast<int>(flags & 0x7fffffffu) : -st;
 }
 
 const char* kvq_strerror(int32_t status) {

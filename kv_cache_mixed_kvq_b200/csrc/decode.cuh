@@ -8,9 +8,11 @@
 //   o   = sum_t softmax(s)_t v^_t
 //
 // Design (B200, sm_100a):
-//  * a producer warp streams 64-token stages of the four cache arrays into
-//    shared memory with 1-D bulk copies (cp.async.bulk, no multicast) on an
-//    mbarrier ring; four consumer warps each take one 16-token tile;
+//  * each of the CTA's four warps runs its own copy pipeline: lane 0 streams
+//    the warp's next 32 positions of the four cache arrays into a ring of
+//    2-3 shared-memory slots with 1-D bulk copies (cp.async.bulk, no
+//    multicast) counted on the warp's own mbarriers (bounded waits), and the
+//    warp processes its two 16-token tiles phase by phase;
 //  * codes stay integers: every code becomes an exact binary16 subnormal
 //    (code * 2^(pos-24)) with one AND, so tensor cores (mma.sync m16n8k16,
 //    fp32 accumulate) multiply raw codes; the per-group scale and zero are
@@ -135,6 +137,33 @@ __device__ __forceinline__ void mma_f16_16816_zc(float d[4], uint32_t a0, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
+// Shared-memory 8x8 b16 matrix stores and transposed loads (N = 2 or 4
+// matrices; each lane addresses one 16-byte row: matrix lane/8, row lane%8).
+template <int N>
+__device__ __forceinline__ void stmatrix_b16(void* p, const uint32_t* r) {
+  if constexpr (N == 4)
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(p)),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+                 : "memory");
+  else
+    asm volatile("stmatrix.sync.aligned.m8n8.x2.shared.b16 [%0], {%1, %2};" ::"r"(smem_addr(p)), "r"(r[0]),
+                 "r"(r[1])
+                 : "memory");
+}
+template <int N>
+__device__ __forceinline__ void ldmatrix_trans_b16(const void* p, uint32_t* d) {
+  if constexpr (N == 4)
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+                 : "r"(smem_addr(p))
+                 : "memory");
+  else
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(d[0]), "=r"(d[1])
+                 : "r"(smem_addr(p))
+                 : "memory");
+}
+
 // (scale, zero) words of two consecutive positions (N groups each).
 template <int N>
 __device__ __forceinline__ void lds_param_pair(const uint32_t* p, uint32_t (&w0)[N], uint32_t (&w1)[N]) {
@@ -171,6 +200,13 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   const int b = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  uint64_t* wfull = full + warp * C::kSlots;
+  if (lane == 0) {
+    for (int sl = 0; sl < C::kSlots; ++sl) mbar_init(&wfull[sl], 1);
+    fence_barrier_init();
+  }
+  pdl_wait();
+  pdl_trigger();
 
   int len = a.seq_lens[b];
   const int lim = min(a.max_seq_len, a.capacity);
@@ -190,7 +226,6 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   // of the split for it = 0 .. my_iters-1, kSlots copies in flight.
   const int my_first = warp * 16 * C::TPW;
   const int my_iters = n_tok > my_first ? (n_tok - my_first + C::kStageTokens - 1) / C::kStageTokens : 0;
-  uint64_t* wfull = full + warp * C::kSlots;
   uint8_t* wring = smem + warp * C::kSlots * C::SLOT_BYTES;
   const uint8_t* kb = a.k_codes + slot * a.capacity * C::KROW;
   const uint8_t* vb = a.v_codes + slot * (a.capacity / 16) * C::VTILE;
@@ -210,11 +245,8 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V + C::SLOT_P, vpb + static_cast<size_t>(tb) * C::PROW,
                   pbytes, &wfull[sl]);
   };
-  if (lane == 0) {
-    for (int sl = 0; sl < C::kSlots; ++sl) mbar_init(&wfull[sl], 1);
-    fence_barrier_init();
+  if (lane == 0)
     for (int it = 0; it < min(C::kSlots, my_iters); ++it) issue(it, it);
-  }
   __syncwarp();
 
   // ------------------------------------------------------------ consumers
@@ -349,15 +381,12 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         const int tix = t_first + tt;
         lds_words<C::KSLICE>(st + k_off + tix * 16 * C::KROW, kw[tt], 0);
         lds_words<C::KSLICE>(st + k_off + (tix * 16 + 8) * C::KROW, kw[tt], C::KW);
-        const uint32_t* kp = reinterpret_cast<const uint32_t*>(st + kp_off + tix * 16 * C::PROW);
-        const uint32_t* vq = reinterpret_cast<const uint32_t*>(st + kp_off + tix * 16 * C::PROW + C::SLOT_P);
-#pragma unroll
-        for (int gr = 0; gr < NG; ++gr) {
-          kpa[tt][gr] = kp[gr];
-          kpb[tt][gr] = kp[8 * NG + gr];
-          vpa[tt][gr] = vq[gr];
-          vpb[tt][gr] = vq[8 * NG + gr];
-        }
+        // (scale, zero) words of rows g and g+8: one vector load per row
+        const uint8_t* kp = st + kp_off + tix * 16 * C::PROW;
+        lds_words<C::PROW>(kp, kpa[tt], 0);
+        lds_words<C::PROW>(kp + 8 * C::PROW, kpb[tt], 0);
+        lds_words<C::PROW>(kp + C::SLOT_P, vpa[tt], 0);
+        lds_words<C::PROW>(kp + C::SLOT_P + 8 * C::PROW, vpb[tt], 0);
       }
       // ---- scores: S^T[token][col] = codes . q'
       float acc[NTL][NG][NQ][4];
@@ -500,7 +529,40 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       // ---- weights p * scale_v * 2^u of rows (g, g+8), binary16 high and
       // low parts, staged so that each B-fragment register is one load;
       // zero term accumulated here.
-      {
+      if constexpr (QS == 2) {
+        // Weight matrix of a tile, per (n-tile pt, group): 16 tokens x 8
+        // columns (head 4pt + c/2 ... : column 2c = high, 2c+1 = low part),
+        // i.e. the score fragment layout itself; stored as two 8x8 b16
+        // matrices (tokens 0-7, 8-15) with one stmatrix per four matrices.
+        const float fu = pow2i(u_run);
+#pragma unroll
+        for (int tt = 0; tt < NTL; ++tt) {
+          uint32_t mr[2 * NG * NP];
+#pragma unroll
+          for (int gr = 0; gr < NG; ++gr) {
+            const float2 sc = scales_of(vpa[tt][gr], vpb[tt][gr]);
+            const float2 zr = zeros_of(vpa[tt][gr], vpb[tt][gr]);
+#pragma unroll
+            for (int hs = 0; hs < HT; ++hs) {
+              const float2 P = __fmul2_rn(__fmul2_rn(pr[tt][hs], make_float2(fu, fu)), sc);
+              const uint32_t hi = f2_to_h2(P.x, P.y);
+              const float2 hf = unpack_half2(hi);
+              const uint32_t lo = f2_to_h2(P.x - hf.x, P.y - hf.y);
+              mr[2 * (hs * NG + gr)] = __byte_perm(hi, lo, 0x5410);      // row g: (high, low)
+              mr[2 * (hs * NG + gr) + 1] = __byte_perm(hi, lo, 0x7632);  // row g + 8
+              zacc[hs][gr] = __ffma2_rn(pr[tt][hs], zr, zacc[hs][gr]);
+            }
+          }
+          uint8_t* wbt = reinterpret_cast<uint8_t*>(wb + (t_first + tt) * C::WB_HALVES);
+#pragma unroll
+          for (int m0 = 0; m0 < 2 * NG * NP; m0 += 4) {
+            if constexpr (2 * NG * NP >= 4)
+              stmatrix_b16<4>(wbt + m0 * 128 + lane * 16, mr + m0);
+            else
+              stmatrix_b16<2>(wbt + m0 * 128 + lane * 16, mr + m0);
+          }
+        }
+      } else {
         const float fu = pow2i(u_run);
 #pragma unroll
         for (int tt = 0; tt < NTL; ++tt) {
@@ -542,15 +604,35 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       uint32_t vw[NTL][C::VW];
 #pragma unroll
       for (int tt = 0; tt < NTL; ++tt) {
-        const uint16_t* rd = wb + (t_first + tt) * C::WB_HALVES + g * C::WB_RS + 2 * c;
+        if constexpr (QS == 2) {
+          // transposed loads give the B fragments (tokens 2c, 2c+1 | +8, +9; column g)
+          const uint8_t* wbt = reinterpret_cast<const uint8_t*>(wb + (t_first + tt) * C::WB_HALVES);
+          uint32_t d[2 * NG * NP];
 #pragma unroll
-        for (int pt = 0; pt < NP; ++pt)
-#pragma unroll
-          for (int gr = 0; gr < NG; ++gr) {
-            const uint16_t* row = rd + (gr * 8 + 4 * pt) * 2 * C::WB_RS;
-            bp[tt][pt][gr][0] = *reinterpret_cast<const uint32_t*>(row);
-            bp[tt][pt][gr][1] = *reinterpret_cast<const uint32_t*>(row + 8);
+          for (int m0 = 0; m0 < 2 * NG * NP; m0 += 4) {
+            if constexpr (2 * NG * NP >= 4)
+              ldmatrix_trans_b16<4>(wbt + m0 * 128 + lane * 16, d + m0);
+            else
+              ldmatrix_trans_b16<2>(wbt + m0 * 128 + lane * 16, d + m0);
           }
+#pragma unroll
+          for (int pt = 0; pt < NP; ++pt)
+#pragma unroll
+            for (int gr = 0; gr < NG; ++gr) {
+              bp[tt][pt][gr][0] = d[2 * (pt * NG + gr)];
+              bp[tt][pt][gr][1] = d[2 * (pt * NG + gr) + 1];
+            }
+        } else {
+          const uint16_t* rd = wb + (t_first + tt) * C::WB_HALVES + g * C::WB_RS + 2 * c;
+#pragma unroll
+          for (int pt = 0; pt < NP; ++pt)
+#pragma unroll
+            for (int gr = 0; gr < NG; ++gr) {
+              const uint16_t* row = rd + (gr * 8 + 4 * pt) * 2 * C::WB_RS;
+              bp[tt][pt][gr][0] = *reinterpret_cast<const uint32_t*>(row);
+              bp[tt][pt][gr][1] = *reinterpret_cast<const uint32_t*>(row + 8);
+            }
+        }
 #pragma unroll
         for (int pc = 0; pc < C::VN / C::VP; ++pc)
           lds_words<C::VP>(st + v_off + (t_first + tt) * C::VTILE + pc * 32 * C::VP, vw[tt],
@@ -687,8 +769,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
 
 template <class C>
 cudaError_t launch_decode(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
-  decode_kernel<C><<<grid, C::kThreads, C::SMEM_BYTES, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(decode_kernel<C>, grid, dim3(C::kThreads), C::SMEM_BYTES, stream, a);
 }
 
 template <class C>

@@ -21,7 +21,8 @@ def _declared():
 def test_header_declares_entry_points():
     names = _declared()
     for n in ("kvq_quantize_append", "kvq_decode_attention", "kvq_cache_bytes",
-              "kvq_decode_workspace_bytes", "kvq_device_error_flags", "kvq_strerror"):
+              "kvq_decode_workspace_bytes", "kvq_device_error_flags", "kvq_last_device_error",
+              "kvq_decode_attention_static", "kvq_strerror"):
         assert n in names
 
 

@@ -1,0 +1,89 @@
+"""Host-side logic of the benchmark, on the CPU: the algorithmic byte counts
+behind every GB/s figure, the max-over-ranks reduction of the timed region
+(world size 2 over gloo), and the reference arm's launch under torchrun
+(rank 0 alone prints one JSON line, the other rank exits 0)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from kv_cache_mixed_kvq_b200 import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_algorithmic_bytes_llama_layer():
+    w = workloads.WORKLOADS["llama3_8b"]
+    n_new, pos, read = bench.step_shape(w, (4, 2))
+    assert n_new == 4096 and pos == [0] * 8 and read == [4096] * 8
+    nb = bench.algorithmic_bytes(w, (4, 2), n_new, read)
+    # per token-head: 128*(4+2)/8 code bytes + 2 groups * (scale, zero) binary16
+    assert nb["per_token_head"] == 96 + 16
+    rows = 8 * 8 * 4096
+    # quantize: bf16 K and V read, packed cache written, positions read
+    assert nb["quantize"] == rows * (2 * 128 * 2 + 112) + 4 * 8 == 163_577_888
+    # decode: every cached token-head once, bf16 Q read and output written, lengths
+    assert nb["decode"] == 8 * 4096 * 8 * 112 + 2 * 8 * 32 * 128 * 2 + 4 * 8 == 29_491_232
+
+
+def test_step_shapes_append_workloads():
+    for name, n in (("long", 1), ("qwen_mistral", 16), ("ragged", 0), ("tiny", 0)):
+        w = workloads.WORKLOADS[name]
+        n_new, pos, read = bench.step_shape(w, w.bits[0])
+        assert n_new == n
+        lens = workloads.seq_lens(w).tolist()
+        assert read == lens
+        assert pos == ([x - n for x in lens] if n else lens)
+        assert max(read) <= w.capacity()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _max_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.max_over_ranks(1.5 + rank, world, torch.device("cpu"))
+        q.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world_2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_max_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = dict(q.get(timeout=5) for _ in range(2))
+    assert got == {0: 2.5, 1: 2.5}
+    assert bench.max_over_ranks(3.0, 1, torch.device("cpu")) == 3.0
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py",
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3",
+           "--workload", "tiny"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    res = json.loads(lines[0])
+    assert res["impl"] == "reference" and res["value"] > 0 and res["unit"] == "GB/s"
+    assert res["cpu_baseline"]["kind"] == "oracle"
+    assert res["e2e"]["h2d_bytes_per_step"] == 0

@@ -130,6 +130,10 @@ def test_length_clamping_flags(ora):
     out, ref = _run(ora, 2, 1, 2, 64, 4, 2, 32, [40, 40], max_len=32, seed=15)
     compare_attention(out, ref)
     assert kvq.kvq_device_error_flags() & kvq.KVQ_DEVERR_SEQ_LEN
+    # the single-value form reads the same word, and reading clears it
+    _run(ora, 2, 1, 2, 64, 4, 2, 32, [40, 40], max_len=32, seed=15)
+    assert kvq.kvq_last_device_error() == kvq.KVQ_DEVERR_SEQ_LEN
+    assert kvq.kvq_last_device_error() == 0
 
 
 def test_workspace_too_small_is_rejected():
