@@ -68,7 +68,8 @@ def _sampled_slots(w, read):
     if w.ragged:
         slots.add((int(np.argmax(read)), 1 % w.kv_heads))
         slots.add((int(np.argmin(read)), 2 % w.kv_heads))
-    while len(slots) < (6 if w.ragged else 4):
+    want = min(6 if w.ragged else 4, w.batch * w.kv_heads)
+    while len(slots) < want:
         slots.add((rng.randrange(w.batch), rng.randrange(w.kv_heads)))
     return sorted(slots)
 
