@@ -78,22 +78,27 @@ def sha_of(paths):
 KERNEL_SOURCES = {
     "quantize": ["kv_cache_mixed_kvq_b200/csrc/quantize.cuh", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
     "decode": ["kv_cache_mixed_kvq_b200/csrc/decode.cuh", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
+    "combine": ["kv_cache_mixed_kvq_b200/csrc/combine.cu", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
 }
 
 
-def measured_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it still
-    matches the kernel source; else None."""
+def measured_traffic(kernels, workload: str):
+    """DRAM bytes per call (sum over `kernels`) from the committed ncu summary
+    (profiles/ncu_traffic.json), if every entry still matches its kernel
+    source; else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             data = json.load(f)
     except (OSError, ValueError):
         return None
-    rec = data.get(f"{kernel}/{workload}")
-    if not rec or rec.get("source_sha") != sha_of(KERNEL_SOURCES[kernel]):
-        return None
-    return rec.get("dram_bytes_per_launch")
+    total = 0
+    for kernel in kernels:
+        rec = data.get(f"{kernel}/{workload}")
+        if not rec or rec.get("source_sha") != sha_of(KERNEL_SOURCES[kernel]):
+            return None
+        total += rec["dram_bytes_per_launch"]
+    return total
 
 
 def peaks():
@@ -284,8 +289,8 @@ def run_ours(args, rank, world, device):
         ach = nbytes[key] / t_s / 1e9
         roof[name] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak,
                       "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
-                      "traffic": measured_traffic("quantize" if key == "quantize" else "decode",
-                                                  w.name),
+                      "traffic": measured_traffic(
+                          ["quantize"] if key == "quantize" else ["decode", "combine"], w.name),
                       "ms": round(kern[name], 5), "algorithmic_bytes": nbytes[key],
                       "peak_source": f"{peak_kind} hbm_gbs (copy)"}
     dominant = "quantize" if "quantize" in roof and kern["quantize"] >= kern.get(

@@ -228,12 +228,13 @@ struct QTile {
   bool bad;  // pos[b] is negative or the append overruns the capacity
 };
 
-__device__ __forceinline__ QTile q_tile(const QuantizeArgs& a, long long idx, int ntps) {
+__device__ __forceinline__ QTile q_tile(const QuantizeArgs& a, int idx) {
   QTile t;
-  t.x = static_cast<int>(idx % ntps);
-  const long long sh = idx / ntps;
-  t.h = static_cast<int>(sh % a.kv_heads);
-  t.b = static_cast<int>(sh / a.kv_heads);
+  const uint32_t sh = fast_div(static_cast<uint32_t>(idx), a.div_ntps);
+  t.x = idx - static_cast<int>(sh) * a.ntps;
+  const uint32_t b = fast_div(sh, a.div_heads);
+  t.h = static_cast<int>(sh - b * a.kv_heads);
+  t.b = static_cast<int>(b);
   t.pos = a.pos[t.b];
   t.bad = t.pos < 0 || static_cast<long long>(t.pos) + a.n_new > a.capacity;
   t.ok = false;
@@ -248,26 +249,48 @@ __device__ __forceinline__ QTile q_tile(const QuantizeArgs& a, long long idx, in
   return t;
 }
 
-// Issues the cp.async copies of tile t's input rows into `stage`: consecutive
-// threads copy consecutive 16-byte pieces of a row (coalesced), each piece
-// landing in the padded chunk of the thread that will quantize it.
+// The 16-byte pieces of a tile's 16 input rows (K and V alike) that one
+// thread copies: pieces q = threadIdx.x + i * THREADS.  Consecutive threads
+// copy consecutive pieces of a row (coalesced); each piece lands in the
+// padded chunk of the thread that will quantize it.  The offsets depend only
+// on the thread, so they are computed once per CTA.
 template <class C, typename TIn>
-__device__ __forceinline__ void q_issue(const QuantizeArgs& a, const QTile& t, uint8_t* stage) {
+struct QCopySlots {
   using Pp = QPipe<C, TIn>;
-  if (!t.ok) return;
-  const size_t slot = static_cast<size_t>(t.b) * a.kv_heads + t.h;
-  // input row of tile row r: slot * n_new + (tile * 16 + r - pos)
-  const long long row0 = static_cast<long long>(slot) * a.n_new + t.tile * 16 - t.pos;
-  const uint8_t* kin = reinterpret_cast<const uint8_t*>(a.k) + row0 * Pp::ROWB;
-  const uint8_t* vin = reinterpret_cast<const uint8_t*>(a.v) + row0 * Pp::ROWB;
-  for (int q = t.r0 * Pp::PPR + threadIdx.x; q < t.r1 * Pp::PPR; q += C::THREADS) {
-    const int r = q / Pp::PPR, c = q % Pp::PPR;
-    cp_async16(stage + (r * C::CK + c / Pp::NPK) * Pp::SK + 16 * (c % Pp::NPK),
-               kin + static_cast<size_t>(q) * 16);
-    cp_async16(stage + Pp::KBYTES + (r * C::CV + c / Pp::NPV) * Pp::SV + 16 * (c % Pp::NPV),
-               vin + static_cast<size_t>(q) * 16);
+  static constexpr int PIECES = 16 * Pp::PPR;
+  static constexpr int N = (PIECES + C::THREADS - 1) / C::THREADS;
+  uint32_t koff[N], voff[N];  // shared-memory offsets within a stage
+  int row[N];                 // tile row of the piece (16: none)
+
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const int q = threadIdx.x + i * C::THREADS;
+      const int r = q / Pp::PPR, c = q % Pp::PPR;
+      row[i] = q < PIECES ? r : 16;
+      koff[i] = (r * C::CK + c / Pp::NPK) * Pp::SK + 16 * (c % Pp::NPK);
+      voff[i] = Pp::KBYTES + (r * C::CV + c / Pp::NPV) * Pp::SV + 16 * (c % Pp::NPV);
+    }
   }
-}
+
+  // Copies the appended rows [r0, r1) of tile t into `stage`.
+  __device__ __forceinline__ void issue(const QuantizeArgs& a, const QTile& t, uint8_t* stage) const {
+    if (!t.ok) return;
+    // input row of tile row r: slot * n_new + (tile * 16 + r - pos)
+    const long long row0 = (static_cast<long long>(t.b) * a.kv_heads + t.h) * a.n_new +
+                           (t.tile * 16 - t.pos);
+    const uint8_t* kin = reinterpret_cast<const uint8_t*>(a.k) + row0 * Pp::ROWB;
+    const uint8_t* vin = reinterpret_cast<const uint8_t*>(a.v) + row0 * Pp::ROWB;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      if (row[i] >= t.r0 && row[i] < t.r1) {
+        const uint32_t g = (threadIdx.x + i * C::THREADS) * 16u;
+        cp_async16(stage + koff[i], kin + g);
+        cp_async16(stage + voff[i], vin + g);
+      }
+    }
+  }
+};
 
 template <class C, typename TIn>
 __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const QuantizeArgs a) {
@@ -283,10 +306,10 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
   pdl_wait();
   pdl_trigger();
 
-  const int ntps = (a.n_new + 30) / 16;  // tiles an append of n_new can touch
-  const long long total = static_cast<long long>(ntps) * a.kv_heads * a.batch;
-  const long long first = blockIdx.x, step = gridDim.x;
-  const int my_n = first < total ? static_cast<int>((total - 1 - first) / step + 1) : 0;
+  const int first = blockIdx.x, step = gridDim.x;
+  const int my_n = first < a.total_tiles ? (a.total_tiles - 1 - first) / step + 1 : 0;
+  QCopySlots<C, TIn> cs;
+  cs.init();
 
   const int t = threadIdx.x;
   const bool is_v = t >= C::KT;  // warp-uniform
@@ -297,7 +320,7 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
 
 #pragma unroll 1
   for (int s = 0; s < Pp::STAGES - 1; ++s) {
-    if (s < my_n) q_issue<C, TIn>(a, q_tile(a, first + s * step, ntps), smem + s * Pp::STAGE);
+    if (s < my_n) cs.issue(a, q_tile(a, first + s * step), smem + s * Pp::STAGE);
     cp_async_commit();
   }
 
@@ -306,14 +329,13 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
     {
       const int ahead = i + Pp::STAGES - 1;
       if (ahead < my_n)
-        q_issue<C, TIn>(a, q_tile(a, first + ahead * step, ntps),
-                        smem + (ahead % Pp::STAGES) * Pp::STAGE);
+        cs.issue(a, q_tile(a, first + ahead * step), smem + (ahead % Pp::STAGES) * Pp::STAGE);
       cp_async_commit();
     }
     cp_async_wait<Pp::STAGES - 1>();
     __syncthreads();  // tile i's rows are in its stage
 
-    const QTile tl = q_tile(a, first + i * step, ntps);
+    const QTile tl = q_tile(a, first + i * step);
     if (tl.bad && tl.x == 0 && tl.h == 0 && t == 0)
       flag_error(a.err, tl.pos < 0 ? KVQ_DEVERR_BAD_POS : KVQ_DEVERR_CAPACITY);
     const bool full_tile = tl.ok && tl.r0 == 0 && tl.r1 == 16;
@@ -441,10 +463,16 @@ cudaError_t launch_q(const QuantizeArgs& a, cudaStream_t stream) {
     if (per_sm < 1) per_sm = 1;
     if (dev < kMaxDevices) per_sm_cache[dev].store(per_sm, std::memory_order_relaxed);
   }
-  const long long total = static_cast<long long>((a.n_new + 30) / 16) * a.kv_heads * a.batch;
+  QuantizeArgs w = a;
+  w.ntps = (a.n_new + 30) / 16;  // tiles an append of n_new can touch
+  const long long total = static_cast<long long>(w.ntps) * a.kv_heads * a.batch;
+  if (total >= (1ll << 31)) return cudaErrorInvalidValue;
+  w.total_tiles = static_cast<int>(total);
+  w.div_ntps = make_fast_div(static_cast<uint32_t>(w.ntps));
+  w.div_heads = make_fast_div(static_cast<uint32_t>(a.kv_heads));
   const long long cap = static_cast<long long>(sms) * per_sm;
   const dim3 grid(static_cast<unsigned>(total < cap ? total : cap));
-  return launch_pdl(quantize_append_kernel<C, TIn>, grid, dim3(C::THREADS), Pp::SMEM, stream, a);
+  return launch_pdl(quantize_append_kernel<C, TIn>, grid, dim3(C::THREADS), Pp::SMEM, stream, w);
 }
 
 // Dispatch over (D, G, bits) for one input type.
