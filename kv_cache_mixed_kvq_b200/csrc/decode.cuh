@@ -59,7 +59,10 @@ struct DecodeCfg {
   static constexpr int SLOT_V = TPW * VTILE;
   static constexpr int SLOT_P = 16 * TPW * PROW;
   static constexpr int SLOT_BYTES = SLOT_K + SLOT_V + 2 * SLOT_P;
-  static constexpr int kSlots = SLOT_BYTES > 6144 ? 2 : 3;  // copies in flight per warp
+  // Copies in flight per warp.  Two slots measured as fast as three or four
+  // on every workload shape (graph replay on B200), with a third less
+  // shared memory.
+  static constexpr int kSlots = 2;
   static constexpr int RING_BYTES = kWarps * kSlots * SLOT_BYTES;
   // staged output weights: per warp and tile [group][head][part][WB_RS halves]
   static constexpr int WB_RS = 24;  // halves per row: 16 positions + pad (conflict-free)

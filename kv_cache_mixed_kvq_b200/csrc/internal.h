@@ -28,31 +28,6 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
 
-// Unsigned division by an invariant divisor d >= 1 for dividends below 2^31,
-// as a multiply-high and a shift (Granlund and Montgomery, "Division by
-// invariant integers using multiplication", 1994): with l = ceil(log2 d) and
-// m = ceil(2^(31+l) / d) < 2^32, n / d = floor(n * m / 2^(31+l)) because
-// the error term n * (m*d - 2^(31+l)) / (d * 2^(31+l)) stays below 1/d.
-struct FastDiv {
-  uint32_t d, mul, shift;
-};
-
-inline FastDiv make_fast_div(uint32_t d) {
-  FastDiv f{d, 0u, 0u};
-  if (d <= 1) return f;
-  uint32_t l = 0;
-  while ((1ull << l) < d) ++l;
-  f.mul = static_cast<uint32_t>(((1ull << (31 + l)) + d - 1) / d);
-  f.shift = l - 1;
-  return f;
-}
-
-#ifdef __CUDACC__
-__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
-  return f.d == 1 ? n : (__umulhi(n, f.mul) >> f.shift);
-}
-#endif
-
 struct QuantizeArgs {
   const void* k;
   const void* v;
@@ -65,10 +40,6 @@ struct QuantizeArgs {
   int n_new;
   int batch, kv_heads, head_dim, capacity, bits_k, bits_v, group;
   uint32_t* err;
-  // filled by the launcher: the tile walk (tiles per slot, total) and the
-  // multiply-shift constants that divide tile indices by ntps and kv_heads
-  int ntps, total_tiles;
-  FastDiv div_ntps, div_heads;
 };
 
 cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream);

@@ -4,11 +4,12 @@
 // keys at b_k bits, values at b_v bits; "Results", "Group-size sensitivity":
 // one scale/zero per group of head_dim elements).
 //
-// A persistent grid walks the 16-position tiles of every (batch row, kv
-// head) slot; each CTA stages the input rows of its next tiles in shared
-// memory with cp.async (16-byte pieces, each warp reading contiguous global
-// memory) several tiles ahead of the one it quantizes.  Inside a tile each
-// thread owns a "chunk" of 8*(16/b) consecutive elements of one token:
+// One CTA handles one 16-position tile of one (batch row, kv head) slot;
+// each thread issues all its 16-byte loads before any arithmetic, and about
+// ten 96-thread CTAs stay resident per SM.  (A persistent grid that staged
+// the next tiles in shared memory with cp.async measured slower on B200:
+// more instructions per tile and fewer resident warps.)
+// Each thread owns a "chunk" of 8*(16/b) consecutive elements of one token:
 // exactly the elements whose codes fill one 32-bit word of each of the four
 // K slices (keys), or one 16-bit half-word of each of eight V lanes (values),
 // so every packed word is built inside one thread without shuffles.
@@ -28,8 +29,6 @@
 // written with 16-byte stores; a tile at the edge of the appended range is
 // written element by element so that positions outside it stay untouched.
 #pragma once
-
-#include <atomic>
 
 #include "common.cuh"
 #include "internal.h"
@@ -74,8 +73,8 @@ struct InPair<__nv_bfloat16> {
     __nv_bfloat162 r = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
     return *reinterpret_cast<raw*>(&r);
   }
-  static __device__ __forceinline__ void lds16(const void* p, raw* out) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
+  static __device__ __forceinline__ void load16(const void* p, raw* out) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
     out[0] = u.x; out[1] = u.y; out[2] = u.z; out[3] = u.w;
   }
   static __device__ __forceinline__ raw zero() { return 0u; }
@@ -96,8 +95,8 @@ struct InPair<__half> {
     __half2 r = __hmax2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
     return *reinterpret_cast<raw*>(&r);
   }
-  static __device__ __forceinline__ void lds16(const void* p, raw* out) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
+  static __device__ __forceinline__ void load16(const void* p, raw* out) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
     out[0] = u.x; out[1] = u.y; out[2] = u.z; out[3] = u.w;
   }
   static __device__ __forceinline__ raw zero() { return 0u; }
@@ -114,8 +113,8 @@ struct InPair<float> {
   static __device__ __forceinline__ raw pmax(raw a, raw b) {
     return make_float2(fmaxf(a.x, b.x), fmaxf(a.y, b.y));
   }
-  static __device__ __forceinline__ void lds16(const void* p, raw* out) {
-    const float4 u = *reinterpret_cast<const float4*>(p);
+  static __device__ __forceinline__ void load16(const void* p, raw* out) {
+    const float4 u = __ldg(reinterpret_cast<const float4*>(p));
     out[0] = make_float2(u.x, u.y);
     out[1] = make_float2(u.z, u.w);
   }
@@ -200,116 +199,30 @@ __device__ __forceinline__ void quantize_chunk(const typename InPair<TIn>::raw (
   }
 }
 
-// Shared-memory staging of the input rows.  A stage holds one tile's K and V
-// rows, stored chunk by chunk (the chunk of thread ti at ti * stride) with 16
-// bytes of padding after each chunk, so that the 16-byte reads of a chunk's
-// owner hit distinct banks across each 8-lane phase.
-template <class C, typename TIn>
-struct QPipe {
-  static constexpr int ES = sizeof(TIn);
-  static constexpr int ROWB = C::D * ES;  // bytes per input row
-  static constexpr int PPR = ROWB / 16;   // 16-byte pieces per row
-  static constexpr int NPK = C::CHK * ES / 16, NPV = C::CHV * ES / 16;  // pieces per chunk
-  static constexpr int SK = 16 * (NPK + 1), SV = 16 * (NPV + 1);       // padded chunk strides
-  static constexpr int KBYTES = 16 * C::CK * SK, VBYTES = 16 * C::CV * SV;
-  static constexpr int STAGE = KBYTES + VBYTES;
-  static constexpr int STAGES = ES == 4 ? 2 : 4;  // tiles in flight per CTA
-  static constexpr int OUT = 16 * C::KROW + C::VTILE + 2 * 16 * C::NG * 4;
-  static constexpr int SMEM = STAGES * STAGE + OUT;
-  static_assert(C::CHK * ES % 16 == 0 && C::CHV * ES % 16 == 0, "chunks of whole pieces");
-  static_assert(STAGE % 16 == 0 && (16 * C::KROW) % 16 == 0 && C::VTILE % 16 == 0, "alignment");
-};
-
-// One tile of the walk: slot (b, h), cache tile index, and the rows [r0, r1)
-// of the tile that the append covers.
-struct QTile {
-  int b, h, x, tile, r0, r1, pos;
-  bool ok;   // the tile has rows to write
-  bool bad;  // pos[b] is negative or the append overruns the capacity
-};
-
-__device__ __forceinline__ QTile q_tile(const QuantizeArgs& a, int idx) {
-  QTile t;
-  const uint32_t sh = fast_div(static_cast<uint32_t>(idx), a.div_ntps);
-  t.x = idx - static_cast<int>(sh) * a.ntps;
-  const uint32_t b = fast_div(sh, a.div_heads);
-  t.h = static_cast<int>(sh - b * a.kv_heads);
-  t.b = static_cast<int>(b);
-  t.pos = a.pos[t.b];
-  t.bad = t.pos < 0 || static_cast<long long>(t.pos) + a.n_new > a.capacity;
-  t.ok = false;
-  t.tile = t.r0 = t.r1 = 0;
-  if (t.bad) return t;
-  t.tile = t.pos / 16 + t.x;
-  const int end = t.pos + a.n_new;
-  if (t.tile * 16 >= end) return t;
-  t.r0 = max(t.tile * 16, t.pos) - t.tile * 16;
-  t.r1 = min(t.tile * 16 + 16, end) - t.tile * 16;
-  t.ok = true;
-  return t;
-}
-
-// The 16-byte pieces of a tile's 16 input rows (K and V alike) that one
-// thread copies: pieces q = threadIdx.x + i * THREADS.  Consecutive threads
-// copy consecutive pieces of a row (coalesced); each piece lands in the
-// padded chunk of the thread that will quantize it.  The offsets depend only
-// on the thread, so they are computed once per CTA.
-template <class C, typename TIn>
-struct QCopySlots {
-  using Pp = QPipe<C, TIn>;
-  static constexpr int PIECES = 16 * Pp::PPR;
-  static constexpr int N = (PIECES + C::THREADS - 1) / C::THREADS;
-  uint32_t koff[N], voff[N];  // shared-memory offsets within a stage
-  int row[N];                 // tile row of the piece (16: none)
-
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-      const int q = threadIdx.x + i * C::THREADS;
-      const int r = q / Pp::PPR, c = q % Pp::PPR;
-      row[i] = q < PIECES ? r : 16;
-      koff[i] = (r * C::CK + c / Pp::NPK) * Pp::SK + 16 * (c % Pp::NPK);
-      voff[i] = Pp::KBYTES + (r * C::CV + c / Pp::NPV) * Pp::SV + 16 * (c % Pp::NPV);
-    }
-  }
-
-  // Copies the appended rows [r0, r1) of tile t into `stage`.
-  __device__ __forceinline__ void issue(const QuantizeArgs& a, const QTile& t, uint8_t* stage) const {
-    if (!t.ok) return;
-    // input row of tile row r: slot * n_new + (tile * 16 + r - pos)
-    const long long row0 = (static_cast<long long>(t.b) * a.kv_heads + t.h) * a.n_new +
-                           (t.tile * 16 - t.pos);
-    const uint8_t* kin = reinterpret_cast<const uint8_t*>(a.k) + row0 * Pp::ROWB;
-    const uint8_t* vin = reinterpret_cast<const uint8_t*>(a.v) + row0 * Pp::ROWB;
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-      if (row[i] >= t.r0 && row[i] < t.r1) {
-        const uint32_t g = (threadIdx.x + i * C::THREADS) * 16u;
-        cp_async16(stage + koff[i], kin + g);
-        cp_async16(stage + voff[i], vin + g);
-      }
-    }
-  }
-};
-
 template <class C, typename TIn>
 __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const QuantizeArgs a) {
   constexpr int D = C::D, G = C::G, NG = C::NG;
   using P = InPair<TIn>;
-  using Pp = QPipe<C, TIn>;
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* sk = smem + Pp::STAGES * Pp::STAGE;
-  uint8_t* sv = sk + 16 * C::KROW;
-  uint32_t* skp = reinterpret_cast<uint32_t*>(sv + C::VTILE);
-  uint32_t* svp = skp + 16 * NG;
+  __shared__ __align__(16) uint8_t sk[16 * C::KROW];
+  __shared__ __align__(16) uint8_t sv[C::VTILE];
+  __shared__ __align__(16) uint32_t skp[16 * NG];
+  __shared__ __align__(16) uint32_t svp[16 * NG];
 
+  const int b = blockIdx.z;
+  const int h = blockIdx.y;
   pdl_wait();
   pdl_trigger();
-
-  const int first = blockIdx.x, step = gridDim.x;
-  const int my_n = first < a.total_tiles ? (a.total_tiles - 1 - first) / step + 1 : 0;
-  QCopySlots<C, TIn> cs;
-  cs.init();
+  const int pos = a.pos[b];
+  if (pos < 0 || static_cast<long long>(pos) + a.n_new > a.capacity) {
+    if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0)
+      flag_error(a.err, pos < 0 ? KVQ_DEVERR_BAD_POS : KVQ_DEVERR_CAPACITY);
+    return;
+  }
+  const int tile = pos / 16 + static_cast<int>(blockIdx.x);
+  const int end = pos + a.n_new;
+  if (tile * 16 >= end) return;
+  const bool full_tile = tile * 16 >= pos && tile * 16 + 16 <= end;
+  const size_t slot = static_cast<size_t>(b) * a.kv_heads + h;
 
   const int t = threadIdx.x;
   const bool is_v = t >= C::KT;  // warp-uniform
@@ -317,162 +230,109 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
   const int chunks = is_v ? C::CV : C::CK;
   const int k = ti / chunks;  // position within the tile
   const int w = ti % chunks;  // chunk index within the row
+  const int p = tile * 16 + k;
+  const bool valid = k < 16 && p >= pos && p < end;
 
-#pragma unroll 1
-  for (int s = 0; s < Pp::STAGES - 1; ++s) {
-    if (s < my_n) cs.issue(a, q_tile(a, first + s * step), smem + s * Pp::STAGE);
-    cp_async_commit();
-  }
-
-#pragma unroll 1
-  for (int i = 0; i < my_n; ++i) {
-    {
-      const int ahead = i + Pp::STAGES - 1;
-      if (ahead < my_n)
-        cs.issue(a, q_tile(a, first + ahead * step), smem + (ahead % Pp::STAGES) * Pp::STAGE);
-      cp_async_commit();
+  if (!is_v) {
+    // ------------------------------------------------------------ keys
+    constexpr int CH = C::CHK;
+    typename P::raw raw[CH / 2];
+    if (valid) {
+      const TIn* src = reinterpret_cast<const TIn*>(a.k) +
+                       (slot * a.n_new + (p - pos)) * D + static_cast<size_t>(CH) * w;
+#pragma unroll
+      for (int i = 0; i < CH / 2 / P::PER16; ++i) P::load16(src + i * 2 * P::PER16, raw + i * P::PER16);
+    } else {
+#pragma unroll
+      for (int i = 0; i < CH / 2; ++i) raw[i] = P::zero();
     }
-    cp_async_wait<Pp::STAGES - 1>();
-    __syncthreads();  // tile i's rows are in its stage
-
-    const QTile tl = q_tile(a, first + i * step);
-    if (tl.bad && tl.x == 0 && tl.h == 0 && t == 0)
-      flag_error(a.err, tl.pos < 0 ? KVQ_DEVERR_BAD_POS : KVQ_DEVERR_CAPACITY);
-    const bool full_tile = tl.ok && tl.r0 == 0 && tl.r1 == 16;
-    const size_t slot = static_cast<size_t>(tl.b) * a.kv_heads + tl.h;
-    const uint8_t* stage = smem + (i % Pp::STAGES) * Pp::STAGE;
-
-    if (tl.ok) {
-      const int p = tl.tile * 16 + k;
-      const bool valid = k < 16 && k >= tl.r0 && k < tl.r1;
-      if (!is_v) {
-        // ------------------------------------------------------------ keys
-        constexpr int CH = C::CHK;
-        typename P::raw raw[CH / 2];
-        if (valid) {
-          const uint8_t* src = stage + ti * Pp::SK;
+    uint32_t acc[8];
+    uint32_t par[CH / G > 0 ? CH / G : 1];
+    quantize_chunk<C::BK, G, CH, TIn>(raw, acc, par);
+    constexpr int NPAR = CH / G > 0 ? CH / G : 1;
+    const bool reports = G > CH ? (w % (G / CH)) == 0 : true;
+    const int first_group = (CH * w) / G;
+    if (full_tile && k < 16) {
 #pragma unroll
-          for (int i2 = 0; i2 < Pp::NPK; ++i2) P::lds16(src + 16 * i2, raw + i2 * P::PER16);
-        } else {
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint32_t*>(sk + k * C::KROW + c * C::KSLICE + 4 * w) =
+            __byte_perm(acc[2 * c], acc[2 * c + 1], 0x5410);
+      if (reports)
 #pragma unroll
-          for (int i2 = 0; i2 < CH / 2; ++i2) raw[i2] = P::zero();
-        }
-        uint32_t acc[8];
-        uint32_t par[CH / G > 0 ? CH / G : 1];
-        quantize_chunk<C::BK, G, CH, TIn>(raw, acc, par);
-        constexpr int NPAR = CH / G > 0 ? CH / G : 1;
-        const bool reports = G > CH ? (w % (G / CH)) == 0 : true;
-        const int first_group = (CH * w) / G;
-        if (full_tile && k < 16) {
+        for (int q = 0; q < NPAR; ++q) skp[k * NG + first_group + q] = par[q];
+    } else if (valid) {
+      uint8_t* row = a.k_codes + (slot * a.capacity + p) * C::KROW;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint32_t*>(sk + k * C::KROW + c * C::KSLICE + 4 * w) =
-                __byte_perm(acc[2 * c], acc[2 * c + 1], 0x5410);
-          if (reports)
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint32_t*>(row + c * C::KSLICE + 4 * w) =
+            __byte_perm(acc[2 * c], acc[2 * c + 1], 0x5410);
+      if (reports)
 #pragma unroll
-            for (int q = 0; q < NPAR; ++q) skp[k * NG + first_group + q] = par[q];
-        } else if (valid) {
-          uint8_t* row = a.k_codes + (slot * a.capacity + p) * C::KROW;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint32_t*>(row + c * C::KSLICE + 4 * w) =
-                __byte_perm(acc[2 * c], acc[2 * c + 1], 0x5410);
-          if (reports)
-#pragma unroll
-            for (int q = 0; q < NPAR; ++q)
-              a.k_params[(slot * a.capacity + p) * NG + first_group + q] = par[q];
-        }
-      } else {
-        // ---------------------------------------------------------- values
-        constexpr int CH = C::CHV;
-        typename P::raw raw[CH / 2];
-        if (valid) {
-          const uint8_t* src = stage + Pp::KBYTES + ti * Pp::SV;
-#pragma unroll
-          for (int i2 = 0; i2 < Pp::NPV; ++i2) P::lds16(src + 16 * i2, raw + i2 * P::PER16);
-        } else {
-#pragma unroll
-          for (int i2 = 0; i2 < CH / 2; ++i2) raw[i2] = P::zero();
-        }
-        uint32_t acc[8];
-        uint32_t par[CH / G > 0 ? CH / G : 1];
-        quantize_chunk<C::BV, G, CH, TIn>(raw, acc, par);
-        constexpr int NPAR = CH / G > 0 ? CH / G : 1;
-        const bool reports = G > CH ? (w % (G / CH)) == 0 : true;
-        const int first_group = (CH * w) / G;
-        // half-word of position k in lane 4g + (k mod 8)/2, word (k/8)*WV + w
-        const int n = 4 * ((k / 8) * C::WV + w) + 2 * (k % 2);
-        const int lane0 = (k % 8) / 2;
-        const int off0 = (n / C::VP) * 32 * C::VP + lane0 * C::VP + (n % C::VP);
-        if (full_tile && k < 16) {
-#pragma unroll
-          for (int g = 0; g < 8; ++g)
-            *reinterpret_cast<uint16_t*>(sv + off0 + 4 * g * C::VP) = static_cast<uint16_t>(acc[g]);
-          if (reports)
-#pragma unroll
-            for (int q = 0; q < NPAR; ++q) svp[k * NG + first_group + q] = par[q];
-        } else if (valid) {
-          uint8_t* gt = a.v_codes + (slot * (a.capacity / 16) + tl.tile) * C::VTILE;
-#pragma unroll
-          for (int g = 0; g < 8; ++g)
-            *reinterpret_cast<uint16_t*>(gt + off0 + 4 * g * C::VP) = static_cast<uint16_t>(acc[g]);
-          if (reports)
-#pragma unroll
-            for (int q = 0; q < NPAR; ++q)
-              a.v_params[(slot * a.capacity + p) * NG + first_group + q] = par[q];
-        }
-      }
+        for (int q = 0; q < NPAR; ++q)
+          a.k_params[(slot * a.capacity + p) * NG + first_group + q] = par[q];
     }
-    __syncthreads();  // the stage is free; a full tile's packed output is complete
-    if (full_tile) {
-      uint4* gk = reinterpret_cast<uint4*>(a.k_codes + (slot * a.capacity + tl.tile * 16) * C::KROW);
-      uint4* gv = reinterpret_cast<uint4*>(a.v_codes + (slot * (a.capacity / 16) + tl.tile) * C::VTILE);
-      uint4* gkp = reinterpret_cast<uint4*>(a.k_params + (slot * a.capacity + tl.tile * 16) * NG);
-      uint4* gvp = reinterpret_cast<uint4*>(a.v_params + (slot * a.capacity + tl.tile * 16) * NG);
-      for (int i2 = t; i2 < 16 * C::KROW / 16; i2 += C::THREADS) gk[i2] = reinterpret_cast<const uint4*>(sk)[i2];
-      for (int i2 = t; i2 < C::VTILE / 16; i2 += C::THREADS) gv[i2] = reinterpret_cast<const uint4*>(sv)[i2];
-      for (int i2 = t; i2 < NG * 4; i2 += C::THREADS) {  // 16 * NG words = 4 * NG uint4
-        gkp[i2] = reinterpret_cast<const uint4*>(skp)[i2];
-        gvp[i2] = reinterpret_cast<const uint4*>(svp)[i2];
-      }
+  } else {
+    // ---------------------------------------------------------- values
+    constexpr int CH = C::CHV;
+    typename P::raw raw[CH / 2];
+    if (valid) {
+      const TIn* src = reinterpret_cast<const TIn*>(a.v) +
+                       (slot * a.n_new + (p - pos)) * D + static_cast<size_t>(CH) * w;
+#pragma unroll
+      for (int i = 0; i < CH / 2 / P::PER16; ++i) P::load16(src + i * 2 * P::PER16, raw + i * P::PER16);
+    } else {
+#pragma unroll
+      for (int i = 0; i < CH / 2; ++i) raw[i] = P::zero();
+    }
+    uint32_t acc[8];
+    uint32_t par[CH / G > 0 ? CH / G : 1];
+    quantize_chunk<C::BV, G, CH, TIn>(raw, acc, par);
+    constexpr int NPAR = CH / G > 0 ? CH / G : 1;
+    const bool reports = G > CH ? (w % (G / CH)) == 0 : true;
+    const int first_group = (CH * w) / G;
+    // half-word of position k in lane 4g + (k mod 8)/2, word (k/8)*WV + w
+    const int n = 4 * ((k / 8) * C::WV + w) + 2 * (k % 2);
+    const int lane0 = (k % 8) / 2;
+    const int off0 = (n / C::VP) * 32 * C::VP + lane0 * C::VP + (n % C::VP);
+    if (full_tile && k < 16) {
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        *reinterpret_cast<uint16_t*>(sv + off0 + 4 * g * C::VP) = static_cast<uint16_t>(acc[g]);
+      if (reports)
+#pragma unroll
+        for (int q = 0; q < NPAR; ++q) svp[k * NG + first_group + q] = par[q];
+    } else if (valid) {
+      uint8_t* gt = a.v_codes + (slot * (a.capacity / 16) + tile) * C::VTILE;
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        *reinterpret_cast<uint16_t*>(gt + off0 + 4 * g * C::VP) = static_cast<uint16_t>(acc[g]);
+      if (reports)
+#pragma unroll
+        for (int q = 0; q < NPAR; ++q)
+          a.v_params[(slot * a.capacity + p) * NG + first_group + q] = par[q];
     }
   }
-  cp_async_wait<0>();  // no copy may land after the CTA has exited
+
+  if (full_tile) {
+    __syncthreads();
+    uint4* gk = reinterpret_cast<uint4*>(a.k_codes + (slot * a.capacity + tile * 16) * C::KROW);
+    uint4* gv = reinterpret_cast<uint4*>(a.v_codes + (slot * (a.capacity / 16) + tile) * C::VTILE);
+    uint4* gkp = reinterpret_cast<uint4*>(a.k_params + (slot * a.capacity + tile * 16) * NG);
+    uint4* gvp = reinterpret_cast<uint4*>(a.v_params + (slot * a.capacity + tile * 16) * NG);
+    for (int i = t; i < 16 * C::KROW / 16; i += C::THREADS) gk[i] = reinterpret_cast<const uint4*>(sk)[i];
+    for (int i = t; i < C::VTILE / 16; i += C::THREADS) gv[i] = reinterpret_cast<const uint4*>(sv)[i];
+    for (int i = t; i < NG * 4; i += C::THREADS) {  // 16 * NG words = 4 * NG uint4
+      gkp[i] = reinterpret_cast<const uint4*>(skp)[i];
+      gvp[i] = reinterpret_cast<const uint4*>(svp)[i];
+    }
+  }
 }
 
-// Persistent launch: as many CTAs as fit on the device at once (queried
-// once per device), each walking tiles blockIdx.x, blockIdx.x + gridDim.x, ...
 template <int D, int BK, int BV, int G, typename TIn>
 cudaError_t launch_q(const QuantizeArgs& a, cudaStream_t stream) {
   using C = QCfg<D, BK, BV, G>;
-  using Pp = QPipe<C, TIn>;
-  constexpr int kMaxDevices = 64;
-  static std::atomic<int> per_sm_cache[kMaxDevices];
-  int dev = 0, sms = 0, per_sm = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  if (dev < kMaxDevices) per_sm = per_sm_cache[dev].load(std::memory_order_relaxed);
-  if (per_sm == 0) {
-    e = cudaFuncSetAttribute(quantize_append_kernel<C, TIn>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, Pp::SMEM);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_append_kernel<C, TIn>,
-                                                        C::THREADS, Pp::SMEM);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) per_sm = 1;
-    if (dev < kMaxDevices) per_sm_cache[dev].store(per_sm, std::memory_order_relaxed);
-  }
-  QuantizeArgs w = a;
-  w.ntps = (a.n_new + 30) / 16;  // tiles an append of n_new can touch
-  const long long total = static_cast<long long>(w.ntps) * a.kv_heads * a.batch;
-  if (total >= (1ll << 31)) return cudaErrorInvalidValue;
-  w.total_tiles = static_cast<int>(total);
-  w.div_ntps = make_fast_div(static_cast<uint32_t>(w.ntps));
-  w.div_heads = make_fast_div(static_cast<uint32_t>(a.kv_heads));
-  const long long cap = static_cast<long long>(sms) * per_sm;
-  const dim3 grid(static_cast<unsigned>(total < cap ? total : cap));
-  return launch_pdl(quantize_append_kernel<C, TIn>, grid, dim3(C::THREADS), Pp::SMEM, stream, w);
+  const dim3 grid((a.n_new + 30) / 16, a.kv_heads, a.batch);
+  return launch_pdl(quantize_append_kernel<C, TIn>, grid, dim3(C::THREADS), 0, stream, a);
 }
 
 // Dispatch over (D, G, bits) for one input type.
