@@ -118,12 +118,14 @@ int variant_of(int heads_per_cta, int q_dtype) {
 }
 
 // Split-K plan.  Tokens per split are a multiple of 64, at least 256 (per-CTA
-// set-up and partial-result traffic).  When one wave of resident CTAs gives
-// every (batch row, kv head, head group) at least four splits, use exactly one
-// wave: splits are rounded up, so the grid never spills into a second wave.
-// Otherwise aim at about four waves, so that the block scheduler can balance
-// ragged lengths.  The plan depends only on the shape, Hq, max_seq_len and
-// the device.
+// set-up and partial-result traffic).  When one wave of resident CTAs could
+// give every (batch row, kv head, head group) at least four splits, give it
+// floor(0.7 * slots / units) splits: a little under one wave, because on B200
+// fewer, longer CTAs (2-3 per SM) beat a full wave of short ones (per-CTA
+// set-up and epilogue are amortised over more tokens; measured on the
+// Llama-3-8B-, Qwen- and long-context shapes).  Otherwise aim at about three
+// waves, so that the block scheduler can balance ragged lengths.  The plan
+// depends only on the shape, Hq, max_seq_len and the device.
 int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
   const int gq = Hq / c->kv_heads;
   p->heads_per_cta = gq < 8 ? gq : 8;
@@ -151,13 +153,13 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
   const long long units = static_cast<long long>(c->batch) * c->kv_heads * p->head_groups;
   const long long slots = static_cast<long long>(sms) * per_sm;
   const long long max64 = (max_seq_len + 63LL) / 64 * 64;
-  const long long per_unit = slots / units;
   long long split;
-  if (per_unit >= 4) {
+  if (slots >= 4 * units) {
+    const long long per_unit = (7 * slots) / (10 * units);
     split = ((max_seq_len + per_unit - 1) / per_unit + 63) / 64 * 64;
   } else {
     const long long work = units * max_seq_len;
-    split = ((work + 4 * slots - 1) / (4 * slots) + 63) / 64 * 64;
+    split = ((work + 3 * slots - 1) / (3 * slots) + 63) / 64 * 64;
   }
   if (split < 256) split = 256;
   if (split > max64) split = max64;
