@@ -62,6 +62,13 @@ def _load(path: str | None = None):
     lib.ora_decode_attention.restype = I
     lib.ora_attention_dense.argtypes = [I, I, I, I, P, P, I, P, I, I, P, ctypes.c_float, P]
     lib.ora_attention_dense.restype = I
+    lib.ora_fwht.argtypes = [P, I]
+    lib.ora_fwht.restype = None
+    lib.ora_quantize_append_ex.argtypes = [I] * 7 + [P] * 6 + [I, P, I, I]
+    lib.ora_quantize_append_ex.restype = I
+    lib.ora_decode_attention_ex.argtypes = [I] * 7 + [P] * 4 + [P, I, I, P, I, ctypes.c_float,
+                                                              I, P]
+    lib.ora_decode_attention_ex.restype = I
     return lib
 
 
@@ -133,9 +140,10 @@ def v_code_place(D: int, bits: int, k: int, d: int):
 class HostCache:
     """Host copies of the four cache arrays in the library's format."""
 
-    def __init__(self, B, Hkv, D, capacity, bits_k, bits_v, group):
+    def __init__(self, B, Hkv, D, capacity, bits_k, bits_v, group, rotate_keys=False):
         self.B, self.Hkv, self.D, self.cap = B, Hkv, D, capacity
         self.bits_k, self.bits_v, self.group = bits_k, bits_v, group
+        self.rotate_keys = bool(rotate_keys)  # keys stored as H k (Walsh-Hadamard)
         slots = B * Hkv
         self.k_codes = np.zeros(slots * capacity * D * bits_k // 8, np.uint8)
         self.v_codes = np.zeros(slots * capacity * D * bits_v // 8, np.uint8)
@@ -154,9 +162,10 @@ class HostCache:
         assert k.shape == (self.B, self.Hkv, n_new, self.D) and v.shape == k.shape
         pos = np.ascontiguousarray(pos, dtype=np.int32)
         dt = DTYPE_CODE[_dtype_of(k, dtype)]
-        r = lib().ora_quantize_append(*self._shape(), _ptr(self.k_codes), _ptr(self.v_codes),
-                                      _ptr(self.k_params), _ptr(self.v_params),
-                                      _ptr(k), _ptr(v), dt, _ptr(pos), n_new)
+        r = lib().ora_quantize_append_ex(*self._shape(), _ptr(self.k_codes), _ptr(self.v_codes),
+                                         _ptr(self.k_params), _ptr(self.v_params),
+                                         _ptr(k), _ptr(v), dt, _ptr(pos), n_new,
+                                         int(self.rotate_keys))
         if r < 0:
             raise ValueError("invalid cache shape")
         return r
@@ -185,14 +194,22 @@ class HostCache:
         assert q.shape == (self.B, Hq, self.D)
         lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
         out = np.zeros((self.B, Hq, self.D), np.float64)
-        r = lib().ora_decode_attention(*self._shape(), _ptr(self.k_codes), _ptr(self.v_codes),
+        r = lib().ora_decode_attention_ex(*self._shape(), _ptr(self.k_codes), _ptr(self.v_codes),
                                        _ptr(self.k_params), _ptr(self.v_params), _ptr(q),
                                        DTYPE_CODE[_dtype_of(q, q_dtype)], Hq, _ptr(lens),
                                        self.cap if max_len is None else max_len,
-                                       float(sm_scale), _ptr(out))
+                                       float(sm_scale), int(self.rotate_keys), _ptr(out))
         if r < 0:
             raise ValueError("invalid shape")
         return out, r
+
+
+def fwht(x) -> np.ndarray:
+    """Unnormalised Walsh-Hadamard transform of a binary32 vector (the oracle's
+    key rotation, same butterfly order and rounding)."""
+    y = np.ascontiguousarray(x, dtype=np.float32).copy()
+    lib().ora_fwht(_ptr(y), y.size)
+    return y
 
 
 def attention_dense(k: np.ndarray, v: np.ndarray, q: np.ndarray, seq_lens, sm_scale: float = 0.0,

@@ -26,6 +26,13 @@
  *     dequantised cache (plain definition of one decode step of attention).
  *   - ora_attention_dense: the same on unquantised K/V (the full-precision
  *     baseline of "Results", "Downstream accuracy").
+ *   - ora_fwht and the *_ex variants: key-only rotation ("Results",
+ *     "Integration with rotation": rotating only the keys in a K4V2 setting
+ *     comes close to K4V4; the page names no transform, the plainest reading
+ *     is a Walsh-Hadamard rotation of each key row along head_dim).  Keys are
+ *     stored as H k (H the unnormalised Sylvester Hadamard matrix, computed
+ *     by the butterfly below in binary32); the query is rotated the same way
+ *     and divided by D, so that (H q / D) . (H k) = q . k.
  *
  * Every function here is pinned by the -m "not gpu" tests (closed forms,
  * brute force, library routines, invariants); none is "parity unpinned".
@@ -185,15 +192,41 @@ static int valid_shape(int D, int cap, int bk, int bv, int G) {
   return 1;
 }
 
+/* In-place unnormalised Walsh-Hadamard transform of n = 2^m binary32 values:
+ * for h = 1, 2, 4, ..., n/2 and every pair (i, i+h) with i & h == 0,
+ * (x[i], x[i+h]) <- (x[i] + x[i+h], x[i] - x[i+h]), each a binary32
+ * operation rounded to nearest even.  The result is H x with
+ * H[i][j] = (-1)^popcount(i & j); the stage order fixes the rounding. */
+void ora_fwht(float* x, int n) {
+  for (int h = 1; h < n; h *= 2)
+    for (int i = 0; i < n; ++i)
+      if ((i & h) == 0) {
+        float a = x[i], b = x[i + h];
+        x[i] = a + b;
+        x[i + h] = a - b;
+      }
+}
+
+/* The same transform in binary64 (used on queries). */
+static void fwht_d(double* x, int n) {
+  for (int h = 1; h < n; h *= 2)
+    for (int i = 0; i < n; ++i)
+      if ((i & h) == 0) {
+        double a = x[i], b = x[i + h];
+        x[i] = a + b;
+        x[i + h] = a - b;
+      }
+}
+
 /* Quantize-append into host copies of the four cache arrays, with the same
  * argument meaning as the library call: k, v are [B][Hkv][n_new][D] of
  * dtype, batch row b writes positions pos[b] .. pos[b]+n_new-1.  A batch row
  * whose range leaves [0, cap) is skipped.  Returns the flags: 1 = past
  * capacity, 8 = negative position; -1 for an invalid shape. */
-int ora_quantize_append(int B, int Hkv, int D, int cap, int bk, int bv, int G,
-                        uint8_t* k_codes, uint8_t* v_codes, uint16_t* k_params,
-                        uint16_t* v_params, const void* k, const void* v,
-                        int dtype, const int32_t* pos, int n_new) {
+int ora_quantize_append_ex(int B, int Hkv, int D, int cap, int bk, int bv, int G,
+                           uint8_t* k_codes, uint8_t* v_codes, uint16_t* k_params,
+                           uint16_t* v_params, const void* k, const void* v,
+                           int dtype, const int32_t* pos, int n_new, int rotate_keys) {
   if (!valid_shape(D, cap, bk, bv, G)) return -1;
   int flags = 0;
   int NG = D / G;
@@ -220,6 +253,7 @@ int ora_quantize_append(int B, int Hkv, int D, int cap, int bk, int bv, int G,
           int bits = which == 0 ? bk : bv;
           uint16_t* params = which == 0 ? k_params : v_params;
           for (int d = 0; d < D; ++d) x[d] = load_elem(in, dtype, src + d);
+          if (which == 0 && rotate_keys) ora_fwht(x, D);
           for (int g = 0; g < NG; ++g) {
             float s32, m32;
             uint16_t s16, z16;
@@ -248,6 +282,14 @@ int ora_quantize_append(int B, int Hkv, int D, int cap, int bk, int bv, int G,
   free(x);
   free(codes);
   return flags;
+}
+
+int ora_quantize_append(int B, int Hkv, int D, int cap, int bk, int bv, int G,
+                        uint8_t* k_codes, uint8_t* v_codes, uint16_t* k_params,
+                        uint16_t* v_params, const void* k, const void* v,
+                        int dtype, const int32_t* pos, int n_new) {
+  return ora_quantize_append_ex(B, Hkv, D, cap, bk, bv, G, k_codes, v_codes, k_params,
+                                v_params, k, v, dtype, pos, n_new, 0);
 }
 
 /* Codes of position p of slot (b, h): which = 0 for K, 1 for V. */
@@ -319,12 +361,12 @@ static void attend(int D, int len, const double* q, const float* k_rows,
  * Batch row b attends to positions [0, min(seq_lens[b], max_len, cap)).
  * sm_scale <= 0 selects 1/sqrt(D).  Returns 2 if a length was clamped,
  * -1 on an invalid shape, else 0. */
-int ora_decode_attention(int B, int Hkv, int D, int cap, int bk, int bv, int G,
-                         const uint8_t* k_codes, const uint8_t* v_codes,
-                         const uint16_t* k_params, const uint16_t* v_params,
-                         const void* q, int q_dtype, int Hq,
-                         const int32_t* seq_lens, int max_len, float sm_scale,
-                         double* out) {
+int ora_decode_attention_ex(int B, int Hkv, int D, int cap, int bk, int bv, int G,
+                            const uint8_t* k_codes, const uint8_t* v_codes,
+                            const uint16_t* k_params, const uint16_t* v_params,
+                            const void* q, int q_dtype, int Hq,
+                            const int32_t* seq_lens, int max_len, float sm_scale,
+                            int rotate_keys, double* out) {
   if (!valid_shape(D, cap, bk, bv, G) || Hq % Hkv) return -1;
   int flags = 0;
   int gq = Hq / Hkv;
@@ -351,6 +393,11 @@ int ora_decode_attention(int B, int Hkv, int D, int cap, int bk, int bv, int G,
         int hq = h * gq + j;
         for (int d = 0; d < D; ++d)
           qd[d] = load_elem(q, q_dtype, ((size_t)b * Hq + hq) * D + d);
+        if (rotate_keys) {
+          /* keys are stored rotated: use H q / D */
+          fwht_d(qd, D);
+          for (int d = 0; d < D; ++d) qd[d] /= (double)D;
+        }
         attend(D, len, qd, kr, vr, scale, out + ((size_t)b * Hq + hq) * D);
       }
       free(kr);
@@ -359,6 +406,16 @@ int ora_decode_attention(int B, int Hkv, int D, int cap, int bk, int bv, int G,
   }
   free(qd);
   return flags;
+}
+
+int ora_decode_attention(int B, int Hkv, int D, int cap, int bk, int bv, int G,
+                         const uint8_t* k_codes, const uint8_t* v_codes,
+                         const uint16_t* k_params, const uint16_t* v_params,
+                         const void* q, int q_dtype, int Hq,
+                         const int32_t* seq_lens, int max_len, float sm_scale,
+                         double* out) {
+  return ora_decode_attention_ex(B, Hkv, D, cap, bk, bv, G, k_codes, v_codes, k_params,
+                                 v_params, q, q_dtype, Hq, seq_lens, max_len, sm_scale, 0, out);
 }
 
 /* Attention on unquantised K/V, [B][Hkv][T][D] of kv_dtype, binary64. */

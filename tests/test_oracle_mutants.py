@@ -15,6 +15,7 @@ from tests import test_oracle_attention as att
 from tests import test_oracle_layout as lay
 from tests import test_oracle_numbers as num
 from tests import test_oracle_quantizer as qz
+from tests import test_oracle_rotation as rot
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "kvq_oracle.c")
 
@@ -35,6 +36,13 @@ MUTANTS = {
     # first occurrence: the packed-cache attention
     "gqa_modulo": ("int hq = h * gq + j;", "int hq = j * Hkv + h;"),
     "f16_ties_away": ("double n = nearbyint(a / spacing);", "double n = round(a / spacing);"),
+    # key-only rotation
+    "fwht_butterfly_swapped": ("        x[i] = a + b;\n        x[i + h] = a - b;",
+                               "        x[i] = a - b;\n        x[i + h] = a + b;"),
+    "rotated_query_not_divided": ("for (int d = 0; d < D; ++d) qd[d] /= (double)D;", ""),
+    "keys_not_rotated": ("if (which == 0 && rotate_keys) ora_fwht(x, D);", ""),
+    "values_rotated_too": ("if (which == 0 && rotate_keys) ora_fwht(x, D);",
+                           "if (rotate_keys) ora_fwht(x, D);"),
 }
 
 PINS = [
@@ -53,6 +61,9 @@ PINS = [
     lambda o: att.test_single_token_returns_its_value(o),
     lambda o: att.test_brute_force_tiny(o, 3),
     lambda o: att.test_library_softmax_gqa(o, 4, 2, 64),
+    lambda o: rot.test_fwht_is_the_sylvester_hadamard_product(o, 64),
+    lambda o: rot.test_rotated_keys_dequantise_near_the_rotated_row(o),
+    lambda o: rot.test_rotated_decode_matches_dense_attention_at_8_bits(o),
 ]
 
 
