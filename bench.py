@@ -172,7 +172,7 @@ class ClockSampler:
 class Arm:
     """Device buffers for R rotating sets of inputs + caches, and the step."""
 
-    def __init__(self, w, bits, rotate: int, device):
+    def __init__(self, w, bits, rotate: int, device, rotate_keys: bool = False):
         import kv_cache_mixed_kvq_b200 as kvq
         self.kvq = kvq
         self.w, self.bits = w, bits
@@ -184,7 +184,8 @@ class Arm:
         self.sets = []
         for r in range(rotate):
             cache = kvq.KVCache.allocate(w.batch, w.kv_heads, w.head_dim, self.cap, bits[0],
-                                         bits[1], w.group, device=device)
+                                         bits[1], w.group, device=device,
+                                         rotate_keys=rotate_keys)
             if w.name != "llama3_8b":
                 # pre-fill the context (untimed); the step then appends n_new tokens
                 for b in range(w.batch):
@@ -225,7 +226,8 @@ def _slot_view(cache, b):
     return type(cache)(1, cache.kv_heads, cache.head_dim, cache.capacity, cache.bits_k,
                        cache.bits_v, cache.group,
                        *[t[b * n:(b + 1) * n] for t, n in zip(
-                           (cache.k_codes, cache.v_codes, cache.k_params, cache.v_params), per)])
+                           (cache.k_codes, cache.v_codes, cache.k_params, cache.v_params), per)],
+                       rotate_keys=cache.rotate_keys)
 
 
 def run_ours(args, rank, world, device):
@@ -233,7 +235,7 @@ def run_ours(args, rank, world, device):
     bits = tuple(int(x) for x in args.bits.split(",")) if args.bits else w.bits[-1] \
         if w.name == "long" else w.bits[0]
     rotate = args.rotate
-    arm = Arm(w, bits, rotate, device)
+    arm = Arm(w, bits, rotate, device, rotate_keys=args.rotate_keys)
     stream = torch.cuda.current_stream()
 
     # warm-up (also loads every kernel and the error-word address)
@@ -314,6 +316,7 @@ def run_ours(args, rank, world, device):
             "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
             "head_dim": w.head_dim, "context": w.context, "input_dtype": w.dtype,
             "bits_k": bits[0], "bits_v": bits[1], "group": w.group,
+            "rotate_keys": bool(args.rotate_keys),
             "step": ("quantize full cache + decode + combine" if w.name == "llama3_8b" else
                      f"append {arm.n_new} + decode + combine"),
             "split_tokens": arm.split_tokens,
@@ -493,6 +496,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--rotate-keys", action="store_true",
+                    help="cache with key-only Walsh-Hadamard rotation (KVQ_FLAG_ROTATE_KEYS)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

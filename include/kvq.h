@@ -127,6 +127,21 @@ enum kvq_device_error {
   KVQ_DEVERR_BAD_POS = 8u      /* pos[b] < 0 (rows skipped)                            */
 };
 
+/* Bits of kvq_cache_desc.flags. */
+enum kvq_cache_flags {
+  /* Key-only rotation (summary page "Quantize What Counts", "Results",
+   * "Integration with rotation": rotating only the keys of a K4V2 cache comes
+   * close to K4V4).  Each key row is stored as H k, H the unnormalised
+   * Walsh-Hadamard matrix of size D (Sylvester order, H[i][j] =
+   * (-1)^popcount(i & j)), computed before quantization by the butterfly
+   * for h = 1, 2, ..., D/2: (x[i], x[i+h]) <- (x[i] + x[i+h], x[i] - x[i+h])
+   * for i & h == 0, each step a binary32 operation rounded to nearest even;
+   * the groups, scales and zeros then apply to H k.  Decode multiplies the
+   * query by H / D, so scores are unchanged in exact arithmetic
+   * ((H q / D) . (H k) = q . k).  Values are never rotated. */
+  KVQ_FLAG_ROTATE_KEYS = 1
+};
+
 /* Which array kvq_cache_bytes() sizes. */
 enum kvq_cache_array {
   KVQ_K_CODES = 0,
@@ -152,7 +167,7 @@ typedef struct kvq_cache_desc {
   int32_t bits_k;
   int32_t bits_v;
   int32_t group;
-  int32_t reserved; /* must be 0 */
+  int32_t flags;    /* kvq_cache_flags; other bits must be 0 */
   uint8_t* k_codes;
   uint8_t* v_codes;
   void* k_params; /* binary16 (scale, zero) pairs */

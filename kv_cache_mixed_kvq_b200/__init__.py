@@ -29,6 +29,7 @@ KVQ_F32, KVQ_BF16, KVQ_F16 = 0, 1, 2
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = range(5)
 KVQ_DEVERR_CAPACITY, KVQ_DEVERR_SEQ_LEN, KVQ_DEVERR_TIMEOUT, KVQ_DEVERR_BAD_POS = 1, 2, 4, 8
 KVQ_K_CODES, KVQ_V_CODES, KVQ_K_PARAMS, KVQ_V_PARAMS = range(4)
+KVQ_FLAG_ROTATE_KEYS = 1
 
 _DTYPE = {torch.float32: KVQ_F32, torch.bfloat16: KVQ_BF16, torch.float16: KVQ_F16}
 
@@ -44,7 +45,7 @@ class KvqCacheDesc(ctypes.Structure):
         ("batch", ctypes.c_int32), ("kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("capacity", ctypes.c_int32),
         ("bits_k", ctypes.c_int32), ("bits_v", ctypes.c_int32),
-        ("group", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("group", ctypes.c_int32), ("flags", ctypes.c_int32),
         ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
         ("k_params", ctypes.c_void_p), ("v_params", ctypes.c_void_p),
     ]
@@ -128,20 +129,23 @@ class KVCache:
     v_codes: torch.Tensor
     k_params: torch.Tensor
     v_params: torch.Tensor
+    rotate_keys: bool = False  # KVQ_FLAG_ROTATE_KEYS: keys stored as H k
 
     @classmethod
     def allocate(cls, batch, kv_heads, head_dim, capacity, bits_k, bits_v, group,
-                 device="cuda") -> "KVCache":
+                 device="cuda", rotate_keys: bool = False) -> "KVCache":
         sizes = [kvq_cache_bytes(batch, kv_heads, head_dim, capacity, bits_k, bits_v, group, w)
                  for w in range(4)]
         if 0 in sizes:
             raise KvqError(KVQ_ERR_INVALID_ARG, "KVCache.allocate")
         bufs = [torch.zeros(n, dtype=torch.uint8, device=device) for n in sizes]
-        return cls(batch, kv_heads, head_dim, capacity, bits_k, bits_v, group, *bufs)
+        return cls(batch, kv_heads, head_dim, capacity, bits_k, bits_v, group, *bufs,
+                   rotate_keys=rotate_keys)
 
     def desc(self) -> KvqCacheDesc:
         return KvqCacheDesc(self.batch, self.kv_heads, self.head_dim, self.capacity,
-                            self.bits_k, self.bits_v, self.group, 0,
+                            self.bits_k, self.bits_v, self.group,
+                            KVQ_FLAG_ROTATE_KEYS if self.rotate_keys else 0,
                             _dev_ptr(self.k_codes, "k_codes"), _dev_ptr(self.v_codes, "v_codes"),
                             _dev_ptr(self.k_params, "k_params"), _dev_ptr(self.v_params, "v_params"))
 

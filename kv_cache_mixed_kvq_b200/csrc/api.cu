@@ -63,7 +63,7 @@ int check_shape(int B, int Hkv, int D, int cap, int bk, int bv, int G) {
 }
 
 int check_cache(const kvq_cache_desc* c) {
-  if (!c || c->reserved != 0) return KVQ_ERR_INVALID_ARG;
+  if (!c || (c->flags & ~KVQ_FLAG_ROTATE_KEYS) != 0) return KVQ_ERR_INVALID_ARG;
   const int st = check_shape(c->batch, c->kv_heads, c->head_dim, c->capacity, c->bits_k,
                              c->bits_v, c->group);
   if (st != KVQ_OK) return st;
@@ -118,14 +118,13 @@ int variant_of(int heads_per_cta, int q_dtype) {
 }
 
 // Split-K plan.  Tokens per split are a multiple of 64, at least 256 (per-CTA
-// set-up and partial-result traffic).  When one wave of resident CTAs could
-// give every (batch row, kv head, head group) at least four splits, give it
-// floor(0.7 * slots / units) splits: a little under one wave, because on B200
-// fewer, longer CTAs (2-3 per SM) beat a full wave of short ones (per-CTA
-// set-up and epilogue are amortised over more tokens; measured on the
-// Llama-3-8B-, Qwen- and long-context shapes).  Otherwise aim at about three
-// waves, so that the block scheduler can balance ragged lengths.  The plan
-// depends only on the shape, Hq, max_seq_len and the device.
+// set-up and partial-result traffic).  When one wave of resident CTAs gives
+// every (batch row, kv head, head group) at least four splits, use exactly
+// one wave: splits are rounded up, so the grid never spills into a second
+// wave, and equal lengths finish together.  Otherwise aim at about three
+// waves, so that the block scheduler can balance ragged lengths (measured on
+// B200 with cold caches: three waves beat four on the ragged batch).  The
+// plan depends only on the shape, Hq, max_seq_len and the device.
 int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
   const int gq = Hq / c->kv_heads;
   p->heads_per_cta = gq < 8 ? gq : 8;
@@ -155,7 +154,7 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
   const long long max64 = (max_seq_len + 63LL) / 64 * 64;
   long long split;
   if (slots >= 4 * units) {
-    const long long per_unit = (7 * slots) / (10 * units);
+    const long long per_unit = slots / units;
     split = ((max_seq_len + per_unit - 1) / per_unit + 63) / 64 * 64;
   } else {
     const long long work = units * max_seq_len;
@@ -256,6 +255,7 @@ int kvq_quantize_append(const kvq_cache_desc* cache, const void* k, const void* 
   a.bits_k = cache->bits_k;
   a.bits_v = cache->bits_v;
   a.group = cache->group;
+  a.rotate_keys = (cache->flags & KVQ_FLAG_ROTATE_KEYS) != 0;
   st = error_word(&a.err);
   if (st != KVQ_OK) return st;
   return to_status(kvq::launch_quantize_append(a, reinterpret_cast<cudaStream_t>(stream)));
@@ -323,6 +323,7 @@ int kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int32_t q_d
     a.split_tokens = p.split_tokens;
     a.num_splits = p.num_splits;
     a.sm_scale_log2 = scale * 1.4426950408889634f;
+    a.rotate_q = (cache->flags & KVQ_FLAG_ROTATE_KEYS) != 0;
     a.ws_o = ws_o;
     a.ws_lse = ws_lse;
     st = error_word(&a.err);

@@ -74,6 +74,7 @@ struct DecodeCfg {
       RING_BYTES + WB_BYTES + 4 * (ALPHA_FLOATS + MERGE_FLOATS) + 8 * kWarps * kSlots;
   static constexpr int HT = QS == 1 ? 2 * NQ : NQ;  // score head slots per lane
   static_assert(RING_BYTES >= kWarps * 8 * D * 4, "merge buffer must fit in the ring");
+  static_assert(WB_BYTES >= 8 * D * 4, "rotated queries must fit in the staging buffer");
   static_assert(SLOT_BYTES % 16 == 0 && SLOT_K % 16 == 0 && SLOT_V % 16 == 0, "alignment");
   static_assert(G >= 16 && G % 16 == 0, "group must cover whole 16-element steps");
 };
@@ -279,6 +280,29 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
 
   {
     // -------- query fragments (B operand of the score product), once per CTA
+    // With rotated keys (KVQ_FLAG_ROTATE_KEYS) the query becomes H q / D: the
+    // CTA's query rows are transformed in shared memory first (the weight
+    // staging buffer is unused until the first tile).
+    const float* qrot = nullptr;
+    if (a.rotate_q) {
+      float* qs = reinterpret_cast<float*>(wbuf);  // [head][D]
+      for (int i = threadIdx.x; i < nh * D; i += C::kThreads)
+        qs[i] = load_elem(a.q, a.q_dtype,
+                          (static_cast<size_t>(b) * a.q_heads + head0 + i / D) * D + i % D);
+      __syncthreads();
+#pragma unroll 1
+      for (int h = 1; h < D; h *= 2) {
+        for (int i = threadIdx.x; i < nh * D / 2; i += C::kThreads) {
+          const int r = i % (D / 2);
+          float* x = qs + (i / (D / 2)) * D + (r / h) * 2 * h + (r % h);
+          const float x0 = x[0], x1 = x[h];
+          x[0] = x0 + x1;
+          x[h] = x0 - x1;
+        }
+        __syncthreads();
+      }
+      qrot = qs;
+    }
     float qraw[NQ][KSTEPS][4];
     float amax = 0.0f;
 #pragma unroll
@@ -293,7 +317,11 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
           // elements d, d+1 with d = 16j + 2c + 8r
           const size_t d = row + 16 * j + 2 * c + 8 * r;
           float2 v = make_float2(0.0f, 0.0f);
-          if (head < nh) {
+          if (head < nh && qrot != nullptr) {
+            constexpr float kInvD = 1.0f / D;  // exact: D is a power of two
+            const float* x = qrot + head * D + 16 * j + 2 * c + 8 * r;
+            v = make_float2(x[0] * kInvD, x[1] * kInvD);
+          } else if (head < nh) {
             if (a.q_dtype == KVQ_F32) {
               v = __ldg(reinterpret_cast<const float2*>(a.q) + d / 2);
             } else {
@@ -308,6 +336,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
           amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
         }
     }
+    if (qrot != nullptr) __syncthreads();  // every warp has read qs before any stages weights
     amax = warp_max_xor(amax, 1);
     const int eq = amax > 0.0f ? max(-100, min(100, 14 - ilogbf(amax))) : 0;
     uint32_t bq[NQ][KSTEPS][2];

@@ -40,6 +40,7 @@ struct QuantizeArgs {
   int n_new;
   int batch, kv_heads, head_dim, capacity, bits_k, bits_v, group;
   uint32_t* err;
+  bool rotate_keys;  // store keys as H k (Walsh-Hadamard along head_dim)
 };
 
 cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream);
@@ -59,6 +60,7 @@ struct DecodeArgs {
   int split_tokens;   // multiple of 64
   int num_splits;     // grid.x
   float sm_scale_log2;  // softmax scale times log2(e)
+  bool rotate_q;        // keys are stored rotated: use H q / D
   float* ws_o;        // [B][Hq][num_splits][D] partial outputs
   float* ws_lse;      // [B][Hq][num_splits] log2-domain log-sum-exp
   uint32_t* err;

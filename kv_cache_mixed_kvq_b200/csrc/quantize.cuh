@@ -199,7 +199,39 @@ __device__ __forceinline__ void quantize_chunk(const typename InPair<TIn>::raw (
   }
 }
 
-template <class C, typename TIn>
+// Walsh-Hadamard transform of a key row held as CK chunks of CH binary32
+// values (chunk w of the row in the lane whose chunk index is w, the row's
+// chunks in consecutive lanes): the butterfly stages h = 1, 2, ..., D/2 in
+// that order, (x[i], x[i+h]) <- (x[i] + x[i+h], x[i] - x[i+h]) for i & h == 0;
+// stages with h < CH stay in the thread, the others exchange with lane xor
+// h/CH (key rotation of the cache format, KVQ_FLAG_ROTATE_KEYS).
+template <int CH, int CK>
+__device__ __forceinline__ void rotate_row_chunk(float2 (&f)[CH / 2], int w) {
+#pragma unroll
+  for (int i = 0; i < CH / 2; ++i) f[i] = make_float2(f[i].x + f[i].y, f[i].x - f[i].y);  // h = 1
+#pragma unroll
+  for (int hh = 1; hh < CH / 2; hh *= 2)  // h = 2 hh
+#pragma unroll
+    for (int i = 0; i < CH / 2; ++i)
+      if ((i & hh) == 0) {
+        const float2 x = f[i], y = f[i + hh];
+        f[i] = make_float2(x.x + y.x, x.y + y.y);
+        f[i + hh] = make_float2(x.x - y.x, x.y - y.y);
+      }
+#pragma unroll
+  for (int m = 1; m < CK; m *= 2) {  // h = m * CH: partner chunk w ^ m
+    const bool upper = (w & m) != 0;
+#pragma unroll
+    for (int i = 0; i < CH / 2; ++i) {
+      const float yx = __shfl_xor_sync(0xffffffffu, f[i].x, m);
+      const float yy = __shfl_xor_sync(0xffffffffu, f[i].y, m);
+      // lower chunk: own + partner; upper chunk: partner (lower index) - own
+      f[i] = upper ? make_float2(yx - f[i].x, yy - f[i].y) : make_float2(f[i].x + yx, f[i].y + yy);
+    }
+  }
+}
+
+template <class C, typename TIn, bool ROT>
 __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const QuantizeArgs a) {
   constexpr int D = C::D, G = C::G, NG = C::NG;
   using P = InPair<TIn>;
@@ -248,7 +280,16 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
     }
     uint32_t acc[8];
     uint32_t par[CH / G > 0 ? CH / G : 1];
-    quantize_chunk<C::BK, G, CH, TIn>(raw, acc, par);
+    if constexpr (ROT) {
+      // rotated keys: quantize H k, computed in binary32 (exact widening first)
+      float2 f[CH / 2];
+#pragma unroll
+      for (int i = 0; i < CH / 2; ++i) f[i] = P::to_f2(raw[i]);
+      rotate_row_chunk<CH, C::CK>(f, w);
+      quantize_chunk<C::BK, G, CH, float>(f, acc, par);
+    } else {
+      quantize_chunk<C::BK, G, CH, TIn>(raw, acc, par);
+    }
     constexpr int NPAR = CH / G > 0 ? CH / G : 1;
     const bool reports = G > CH ? (w % (G / CH)) == 0 : true;
     const int first_group = (CH * w) / G;
@@ -332,7 +373,9 @@ template <int D, int BK, int BV, int G, typename TIn>
 cudaError_t launch_q(const QuantizeArgs& a, cudaStream_t stream) {
   using C = QCfg<D, BK, BV, G>;
   const dim3 grid((a.n_new + 30) / 16, a.kv_heads, a.batch);
-  return launch_pdl(quantize_append_kernel<C, TIn>, grid, dim3(C::THREADS), 0, stream, a);
+  if (a.rotate_keys)
+    return launch_pdl(quantize_append_kernel<C, TIn, true>, grid, dim3(C::THREADS), 0, stream, a);
+  return launch_pdl(quantize_append_kernel<C, TIn, false>, grid, dim3(C::THREADS), 0, stream, a);
 }
 
 // Dispatch over (D, G, bits) for one input type.
