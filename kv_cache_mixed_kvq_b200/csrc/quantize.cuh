@@ -204,7 +204,14 @@ __device__ __forceinline__ void quantize_chunk(const typename InPair<TIn>::raw (
 // chunks in consecutive lanes): the butterfly stages h = 1, 2, ..., D/2 in
 // that order, (x[i], x[i+h]) <- (x[i] + x[i+h], x[i] - x[i+h]) for i & h == 0;
 // stages with h < CH stay in the thread, the others exchange with lane xor
-// h/CH (key rotation of the cache format, KVQ_FLAG_ROTATE_KEYS).
+// h/CH (key rotation of the cache format, KVQ_FLAG_ROTATE_KEYS).  Stages
+// h >= 2 pair whole float2s and use the packed add; a - b is computed as
+// a + (-b) (the same IEEE operation), the negation a sign flip.
+__device__ __forceinline__ float2 neg2(float2 a) {
+  return make_float2(__uint_as_float(__float_as_uint(a.x) ^ 0x80000000u),
+                     __uint_as_float(__float_as_uint(a.y) ^ 0x80000000u));
+}
+
 template <int CH, int CK>
 __device__ __forceinline__ void rotate_row_chunk(float2 (&f)[CH / 2], int w) {
 #pragma unroll
@@ -215,18 +222,18 @@ __device__ __forceinline__ void rotate_row_chunk(float2 (&f)[CH / 2], int w) {
     for (int i = 0; i < CH / 2; ++i)
       if ((i & hh) == 0) {
         const float2 x = f[i], y = f[i + hh];
-        f[i] = make_float2(x.x + y.x, x.y + y.y);
-        f[i + hh] = make_float2(x.x - y.x, x.y - y.y);
+        f[i] = add2_rn(x, y);
+        f[i + hh] = add2_rn(x, neg2(y));
       }
 #pragma unroll
   for (int m = 1; m < CK; m *= 2) {  // h = m * CH: partner chunk w ^ m
     const bool upper = (w & m) != 0;
 #pragma unroll
     for (int i = 0; i < CH / 2; ++i) {
-      const float yx = __shfl_xor_sync(0xffffffffu, f[i].x, m);
-      const float yy = __shfl_xor_sync(0xffffffffu, f[i].y, m);
+      const float2 y = make_float2(__shfl_xor_sync(0xffffffffu, f[i].x, m),
+                                   __shfl_xor_sync(0xffffffffu, f[i].y, m));
       // lower chunk: own + partner; upper chunk: partner (lower index) - own
-      f[i] = upper ? make_float2(yx - f[i].x, yy - f[i].y) : make_float2(f[i].x + yx, f[i].y + yy);
+      f[i] = add2_rn(y, upper ? neg2(f[i]) : f[i]);
     }
   }
 }
