@@ -303,6 +303,7 @@ def run_ours(args, rank, world, device):
     if not args.no_e2e:
         e2e = run_e2e(arm, args, step_bytes, world, device)
 
+    probe = read_probe_gbs(device)
     result = {
         "metric": METRIC,
         "value": round(world * step_bytes / (ms_step / 1e3) / 1e9, 2),
@@ -326,6 +327,8 @@ def run_ours(args, rank, world, device):
         },
         "kv_tokens_per_s": round(world * nbytes["tokens"] / (ms_step / 1e3), 1),
         "roofline": dict(roof[dominant], kernel=dominant),
+        "read_probe": {"value": probe, "unit": "GB/s",
+                       "what": "torch sum over 1 GiB fp32, best of 10 (context, not the peak)"},
         "roofline_by_kernel": roof,
         "gpu_launches": arm.launches_per_step * args.steps,
         "device_error_flags": flags,
@@ -340,6 +343,25 @@ def run_ours(args, rank, world, device):
         for g in graphs:
             del g
     return result
+
+
+def read_probe_gbs(device, nbytes=1 << 30, reps=10):
+    """HBM read bandwidth of a plain reduction over a 1 GiB buffer (torch's
+    own kernel, best of `reps`): context for the read-only decode, next to
+    the copy bandwidth the roofline divides by."""
+    x = torch.ones(nbytes // 4, dtype=torch.float32, device=device)
+    x.sum()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        x.sum()
+        b.record()
+        torch.cuda.synchronize()
+        best = min(best, a.elapsed_time(b))
+    del x
+    return round(nbytes / (best / 1e3) / 1e9, 1)
 
 
 def per_kernel_times(arm, rotate, stream, reps):
