@@ -188,6 +188,80 @@ __device__ __forceinline__ void lds_param_pair(const uint32_t* p, uint32_t (&w0)
   }
 }
 
+// One attention output element in the caller's type.
+__device__ __forceinline__ void store_out(void* out, int dtype, size_t i, float v) {
+  if (dtype == KVQ_F32)
+    reinterpret_cast<float*>(out)[i] = v;
+  else if (dtype == KVQ_BF16)
+    reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<__half*>(out)[i] = __float2half_rn(v);
+}
+
+// Arrival of one CTA at its unit's counter (epoch << 32 | arrivals): entries
+// of another epoch count as zero.  Returns true for the expected-th arrival.
+// The compare-and-swap retries are bounded; giving up flags a timeout.
+__device__ __forceinline__ bool arrive_last(unsigned long long* ctr, uint32_t epoch, int expected,
+                                            uint32_t* err) {
+  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(ctr);
+  for (int tries = 0; tries < (1 << 20); ++tries) {
+    const unsigned long long assumed = old;
+    const uint32_t n = (static_cast<uint32_t>(assumed >> 32) == epoch
+                            ? static_cast<uint32_t>(assumed) : 0u) + 1u;
+    old = atomicCAS(ctr, assumed, (static_cast<unsigned long long>(epoch) << 32) | n);
+    if (old == assumed) return n == static_cast<uint32_t>(expected);
+  }
+  flag_error(err, KVQ_DEVERR_TIMEOUT);
+  return false;
+}
+
+// Log-sum-exp merge of the ns (<= 16) partial results of the CTA's nh query
+// heads, by the last CTA of the unit to finish: warps take heads, lanes own
+// D/32 output elements, all partial outputs of a lane are requested at once
+// (L2 reads: the other CTAs wrote them just before).
+template <int D, int kWarps>
+__device__ __forceinline__ void merge_partials(const DecodeArgs& a, int b, int head0, int nh,
+                                               int ns) {
+  constexpr int PER = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int h = warp; h < nh; h += kWarps) {
+    const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + h) * a.num_splits;
+    const float lse = lane < ns ? __ldcg(a.ws_lse + row + lane) : -INFINITY;
+    float M = lse;
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+    const float wl = lane < ns ? exp2_approx(lse - M) : 0.0f;
+    float den = wl;
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) den += __shfl_xor_sync(0xffffffffu, den, m);
+    float acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
+#pragma unroll
+    for (int sp = 0; sp < 16; ++sp) {
+      const float w = __shfl_sync(0xffffffffu, wl, sp);
+      if (sp < ns) {
+        const float* o = a.ws_o + (row + sp) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 t = __ldcg(reinterpret_cast<const float4*>(o));
+          acc[0] = fmaf(w, t.x, acc[0]);
+          acc[1] = fmaf(w, t.y, acc[1]);
+          acc[2] = fmaf(w, t.z, acc[2]);
+          acc[3] = fmaf(w, t.w, acc[3]);
+        } else {
+          const float2 t = __ldcg(reinterpret_cast<const float2*>(o));
+          acc[0] = fmaf(w, t.x, acc[0]);
+          acc[1] = fmaf(w, t.y, acc[1]);
+        }
+      }
+    }
+    const float inv = 1.0f / den;
+    const size_t o = (static_cast<size_t>(b) * a.q_heads + head0 + h) * D + lane * PER;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) store_out(a.out, a.out_dtype, o + i, acc[i] * inv);
+  }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a) {
   constexpr int D = C::D, NG = C::NG, NQ = C::NQ, NP = C::NP, QS = C::QS, HT = C::HT;
@@ -219,11 +293,18 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     len = max(0, min(len, lim));
   }
   const int t0 = split * a.split_tokens;
-  if (t0 >= len) return;
-  const int t1 = min(t0 + a.split_tokens, len);
-  const int n_tok = t1 - t0;
   const int head0 = hk * a.gq + hg * a.heads_per_cta;
   const int nh = min(a.heads_per_cta, a.gq - hg * a.heads_per_cta);
+  if (t0 >= len) {
+    // an empty sequence attends to nothing: its output rows are zero
+    if (a.fused && len == 0 && split == 0)
+      for (int i = threadIdx.x; i < nh * D; i += C::kThreads)
+        store_out(a.out, a.out_dtype,
+                  (static_cast<size_t>(b) * a.q_heads + head0 + i / D) * D + i % D, 0.0f);
+    return;
+  }
+  const int t1 = min(t0 + a.split_tokens, len);
+  const int n_tok = t1 - t0;
   const size_t slot = static_cast<size_t>(b) * a.kv_heads + hk;
 
   // ---- this warp's copy pipeline: positions [it*kStageTokens + 16*TPW*warp, +16*TPW)
@@ -727,6 +808,9 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   }
 
   // ------------------------------------------------------------ epilogue
+  // splits with tokens for this batch row; with one, this CTA's result is final
+  const int ns_b = (len + a.split_tokens - 1) / a.split_tokens;
+  const bool direct = a.fused && ns_b == 1;
   __syncthreads();  // all stages consumed; the ring becomes the merge buffer
   float* ob = reinterpret_cast<float*>(smem);  // [warp][8][D]
   float* mb = mrg;                             // [warp][8]
@@ -784,8 +868,10 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       den = fmaf(x, lb[w * 8 + head], den);
     }
     rden[head] = __frcp_rn(den);
-    const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * a.num_splits + split;
-    a.ws_lse[row] = M + __log2f(den);
+    if (!direct) {
+      const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * a.num_splits + split;
+      a.ws_lse[row] = M + __log2f(den);
+    }
   }
   __syncthreads();
   for (int idx = threadIdx.x; idx < nh * D; idx += C::kThreads) {
@@ -794,8 +880,32 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
 #pragma unroll
     for (int w = 0; w < C::kWarps; ++w)
       num = fmaf(wt[head * C::kWarps + w], ob[(w * 8 + head) * D + d] + zb[(w * 8 + head) * NG + d / G], num);
-    const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * a.num_splits + split;
-    a.ws_o[row * D + d] = num * rden[head];
+    if (direct) {
+      store_out(a.out, a.out_dtype, (static_cast<size_t>(b) * a.q_heads + head0 + head) * D + d,
+                num * rden[head]);
+    } else {
+      const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * a.num_splits + split;
+      a.ws_o[row * D + d] = num * rden[head];
+    }
+  }
+  if (a.fused && ns_b > 1) {
+    // publish this split, then the last CTA of the unit merges all of them
+    __threadfence();
+    __syncthreads();
+    int* s_last = reinterpret_cast<int*>(rden + 8);
+    if (threadIdx.x == 0) {
+      unsigned long long* ctr = a.counters + (static_cast<size_t>(b) * gridDim.y + blockIdx.y);
+      const bool last = arrive_last(ctr, a.epoch, ns_b, a.err);
+      *s_last = last;
+    }
+    __syncthreads();
+    if (*s_last) {
+      __threadfence();
+      merge_partials<D, C::kWarps>(a, b, head0, nh, ns_b);
+      if (threadIdx.x == 0)
+        a.counters[static_cast<size_t>(b) * gridDim.y + blockIdx.y] =
+            static_cast<unsigned long long>(a.epoch) << 32;
+    }
   }
 }
 
