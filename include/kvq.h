@@ -213,7 +213,8 @@ int kvq_quantize_append(const kvq_cache_desc* cache, const void* k,
 /*
  * Workspace bytes kvq_decode_attention() needs for this cache, number of
  * query heads and maximum length, on the current device (the split-K plan
- * depends on its SM count).  0 if the arguments are invalid.
+ * depends on its SM count).  0 if the arguments are invalid, and 0 when
+ * every row fits in one split (no workspace is needed then).
  */
 size_t kvq_decode_workspace_bytes(const kvq_cache_desc* cache,
                                   int32_t num_q_heads, int32_t max_seq_len);
@@ -231,12 +232,20 @@ size_t kvq_decode_workspace_bytes(const kvq_cache_desc* cache,
  *   sm_scale    : softmax scale; <= 0 selects 1/sqrt(D).
  *   out         : device, [B][Hq][D], out_dtype in {F32, BF16, F16}.
  *   workspace   : device scratch of at least kvq_decode_workspace_bytes(),
- *                 16-byte aligned; holds per-split partial outputs.
+ *                 16-byte aligned (may be NULL when that is 0); holds the
+ *                 per-split partial outputs and, when the splits are merged
+ *                 inside the decode kernel, one 64-bit arrival counter per
+ *                 (batch row, kv head, head group).  Its contents need no
+ *                 initialisation: counters are tagged with a per-call epoch
+ *                 and reset by the call that used them.  One workspace must
+ *                 not serve two calls that can run concurrently.
  *
- * Two kernel launches on `stream`: split-K flash-decoding over the packed
- * cache, then a log-sum-exp combine of the splits.  Arithmetic: codes are
- * exact in binary16, products and sums in binary32 (tensor cores), softmax
- * in binary32.
+ * Kernel launches on `stream`: split-K flash-decoding over the packed cache,
+ * whose last CTA per (batch row, kv head) merges up to 16 splits with the
+ * log-sum-exp identity (a single split writes the output directly); rows
+ * with more splits are merged by a second, log-sum-exp combine kernel.
+ * Arithmetic: codes are exact in binary16, products and sums in binary32
+ * (tensor cores), softmax in binary32.
  */
 int kvq_decode_attention(const kvq_cache_desc* cache, const void* q,
                          int32_t q_dtype, int32_t num_q_heads,

@@ -137,12 +137,27 @@ def test_length_clamping_flags(ora):
 
 
 def test_workspace_too_small_is_rejected():
-    cache = kvq.KVCache.allocate(1, 1, 128, 64, 4, 2, 64)
+    # 4096 tokens for one (batch row, kv head): several splits, so partial
+    # results (and arrival counters) need a workspace
+    cache = kvq.KVCache.allocate(1, 1, 128, 4096, 4, 2, 64)
     q = torch.zeros(1, 4, 128, dtype=torch.bfloat16, device="cuda")
-    lens = torch.tensor([64], dtype=torch.int32, device="cuda")
-    need = kvq.kvq_decode_workspace_bytes(cache, 4, 64)
+    lens = torch.tensor([4096], dtype=torch.int32, device="cuda")
+    assert kvq.kvq_decode_split_tokens(cache, 4, 4096) < 4096
+    need = kvq.kvq_decode_workspace_bytes(cache, 4, 4096)
     assert need > 0
     ws = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
     with pytest.raises(kvq.KvqError) as e:
-        kvq.kvq_decode_attention(cache, q, lens, 64, workspace=ws)
+        kvq.kvq_decode_attention(cache, q, lens, 4096, workspace=ws)
     assert e.value.status == kvq.KVQ_ERR_WORKSPACE
+
+
+def test_single_split_needs_no_workspace():
+    # one split per row: each CTA writes its rows' final output directly
+    cache = kvq.KVCache.allocate(1, 1, 128, 64, 4, 2, 64)
+    assert kvq.kvq_decode_split_tokens(cache, 4, 64) == 64
+    assert kvq.kvq_decode_workspace_bytes(cache, 4, 64) == 0
+    q = torch.zeros(1, 4, 128, dtype=torch.bfloat16, device="cuda")
+    lens = torch.tensor([64], dtype=torch.int32, device="cuda")
+    out = kvq.kvq_decode_attention(cache, q, lens, 64)  # no workspace
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
