@@ -201,6 +201,8 @@ class Arm:
         self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
         self.split_tokens = kvq.kvq_decode_split_tokens(self.sets[0]["cache"], w.q_heads,
                                                         self.max_len)
+        # one split per row: the decode writes the output, no combine launch
+        self.num_splits = -(-self.max_len // self.split_tokens)
 
     def quantize(self, r):
         s = self.sets[r]
@@ -216,7 +218,8 @@ class Arm:
         self.quantize(r)
         self.decode(r)
 
-    launches_per_step = property(lambda self: (1 if self.n_new else 0) + 2)
+    launches_per_step = property(
+        lambda self: (1 if self.n_new else 0) + (1 if self.num_splits == 1 else 2))
 
 
 def _slot_view(cache, b):

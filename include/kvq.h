@@ -233,17 +233,11 @@ size_t kvq_decode_workspace_bytes(const kvq_cache_desc* cache,
  *   out         : device, [B][Hq][D], out_dtype in {F32, BF16, F16}.
  *   workspace   : device scratch of at least kvq_decode_workspace_bytes(),
  *                 16-byte aligned (may be NULL when that is 0); holds the
- *                 per-split partial outputs and, when the splits are merged
- *                 inside the decode kernel, one 64-bit arrival counter per
- *                 (batch row, kv head, head group).  Its contents need no
- *                 initialisation: counters are tagged with a per-call epoch
- *                 and reset by the call that used them.  One workspace must
- *                 not serve two calls that can run concurrently.
+ *                 per-split partial outputs and log-sum-exps.
  *
  * Kernel launches on `stream`: split-K flash-decoding over the packed cache,
- * whose last CTA per (batch row, kv head) merges up to 16 splits with the
- * log-sum-exp identity (a single split writes the output directly); rows
- * with more splits are merged by a second, log-sum-exp combine kernel.
+ * then a log-sum-exp combine of the splits; when every row fits in one
+ * split, the decode kernel writes the output itself (one launch).
  * Arithmetic: codes are exact in binary16, products and sums in binary32
  * (tensor cores), softmax in binary32.
  */

@@ -2,7 +2,6 @@
 // split-K plan, kernel selection and launches.  No allocation anywhere.
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <map>
@@ -109,16 +108,11 @@ cudaError_t prepare_kernel(const DecodeKernel& k) {
   return e;
 }
 
-// Rows with at most this many splits are merged inside the decode kernel by
-// the last CTA of each (batch row, kv head, head group); longer rows use the
-// separate combine kernel (its merge spreads over more threads).
-constexpr int kFuseMaxSplits = 16;
-
 struct Plan {
   int heads_per_cta, head_groups, split_tokens, num_splits;
-  bool fused;          // merge in the decode kernel (no combine launch)
+  bool direct;         // one split per row: the decode writes the output itself
   size_t ws_o_floats;  // partial outputs [B][Hq][splits][D]
-  size_t ws_bytes;     // partials + log-sum-exps (+ arrival counters when fused)
+  size_t ws_bytes;     // partials + log-sum-exps
 };
 
 int variant_of(int heads_per_cta, int q_dtype) {
@@ -141,7 +135,7 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
   if (max_seq_len <= 0) {
     p->split_tokens = 64;
     p->num_splits = 0;
-    p->fused = false;
+    p->direct = false;
     p->ws_o_floats = 0;
     p->ws_bytes = 0;
     return KVQ_OK;
@@ -179,14 +173,12 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
   p->split_tokens = static_cast<int>(split);
   p->num_splits = static_cast<int>((max_seq_len + split - 1) / split);
   if (p->num_splits > 65535) return KVQ_ERR_UNSUPPORTED;
-  p->fused = p->num_splits <= kFuseMaxSplits;
+  p->direct = p->num_splits == 1;
   p->ws_o_floats = static_cast<size_t>(c->batch) * Hq * p->num_splits * c->head_dim;
-  if (p->num_splits == 1) {
+  if (p->direct) {
     p->ws_bytes = 0;  // every CTA writes its rows' final output
   } else {
     p->ws_bytes = static_cast<size_t>(c->batch) * Hq * p->num_splits * (c->head_dim + 1) * 4;
-    p->ws_bytes = (p->ws_bytes + 15) / 16 * 16;
-    if (p->fused) p->ws_bytes += static_cast<size_t>(units) * 8;  // one 64-bit counter per unit
     p->ws_bytes = (p->ws_bytes + 15) / 16 * 16;
   }
   return KVQ_OK;
@@ -315,12 +307,6 @@ int kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int32_t q_d
   const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf(static_cast<float>(D));
   float* ws_o = p.ws_bytes > 0 ? static_cast<float*>(workspace) : nullptr;
   float* ws_lse = ws_o ? ws_o + p.ws_o_floats : nullptr;
-  unsigned long long* counters = nullptr;
-  if (ws_o && p.fused) {
-    const size_t lse_bytes = (static_cast<size_t>(cache->batch) * num_q_heads * p.num_splits *
-                                  (D + 1) * 4 + 15) / 16 * 16;
-    counters = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + lse_bytes);
-  }
   if (p.num_splits > 0) {
     DecodeKernel k;
     if (!kvq::get_decode_kernel(D, cache->bits_k, cache->bits_v, D / cache->group,
@@ -349,23 +335,14 @@ int kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int32_t q_d
     a.rotate_q = (cache->flags & KVQ_FLAG_ROTATE_KEYS) != 0;
     a.ws_o = ws_o;
     a.ws_lse = ws_lse;
-    a.fused = p.fused;
+    a.direct = p.direct;
     a.out = out;
     a.out_dtype = out_dtype;
-    a.counters = counters;
-    // Arrival counters hold (epoch, count); a call counts only entries of its
-    // own epoch, so the workspace needs no initialisation, and the merging
-    // CTA resets its entry to (epoch, 0), so CUDA-graph replays of one call
-    // (same epoch) also start from zero.
-    static std::atomic<uint32_t> epoch_source{0};
-    uint32_t epoch = ++epoch_source;
-    if (epoch == 0) epoch = ++epoch_source;
-    a.epoch = epoch;
     st = error_word(&a.err);
     if (st != KVQ_OK) return st;
     const dim3 grid(p.num_splits, cache->kv_heads * p.head_groups, cache->batch);
     if (k.launch(a, grid, s) != cudaSuccess) return KVQ_ERR_CUDA;
-    if (p.fused) return KVQ_OK;
+    if (p.direct) return KVQ_OK;
   }
   kvq::CombineArgs ca;
   ca.ws_o = ws_o;

@@ -198,70 +198,6 @@ __device__ __forceinline__ void store_out(void* out, int dtype, size_t i, float 
     reinterpret_cast<__half*>(out)[i] = __float2half_rn(v);
 }
 
-// Arrival of one CTA at its unit's counter (epoch << 32 | arrivals): entries
-// of another epoch count as zero.  Returns true for the expected-th arrival.
-// The compare-and-swap retries are bounded; giving up flags a timeout.
-__device__ __forceinline__ bool arrive_last(unsigned long long* ctr, uint32_t epoch, int expected,
-                                            uint32_t* err) {
-  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(ctr);
-  for (int tries = 0; tries < (1 << 20); ++tries) {
-    const unsigned long long assumed = old;
-    const uint32_t n = (static_cast<uint32_t>(assumed >> 32) == epoch
-                            ? static_cast<uint32_t>(assumed) : 0u) + 1u;
-    old = atomicCAS(ctr, assumed, (static_cast<unsigned long long>(epoch) << 32) | n);
-    if (old == assumed) return n == static_cast<uint32_t>(expected);
-  }
-  flag_error(err, KVQ_DEVERR_TIMEOUT);
-  return false;
-}
-
-// Log-sum-exp merge of the ns (<= 16) partial results of the CTA's nh query
-// heads, by the last CTA of the unit to finish: warps take heads, lanes own
-// D/32 output elements, all partial outputs of a lane are requested at once
-// (L2 reads: the other CTAs wrote them just before).
-template <int D, int kWarps>
-__device__ __forceinline__ void merge_partials(const DecodeArgs& a, int b, int head0, int nh,
-                                               int ns) {
-  constexpr int PER = D / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int h = warp; h < nh; h += kWarps) {
-    const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + h) * a.num_splits;
-    const float lse = lane < ns ? __ldcg(a.ws_lse + row + lane) : -INFINITY;
-    float M = lse;
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
-    const float wl = lane < ns ? exp2_approx(lse - M) : 0.0f;
-    float den = wl;
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1) den += __shfl_xor_sync(0xffffffffu, den, m);
-    float acc[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
-#pragma unroll
-    for (int sp = 0; sp < 16; ++sp) {
-      const float w = __shfl_sync(0xffffffffu, wl, sp);
-      if (sp < ns) {
-        const float* o = a.ws_o + (row + sp) * D + lane * PER;
-        if constexpr (PER == 4) {
-          const float4 t = __ldcg(reinterpret_cast<const float4*>(o));
-          acc[0] = fmaf(w, t.x, acc[0]);
-          acc[1] = fmaf(w, t.y, acc[1]);
-          acc[2] = fmaf(w, t.z, acc[2]);
-          acc[3] = fmaf(w, t.w, acc[3]);
-        } else {
-          const float2 t = __ldcg(reinterpret_cast<const float2*>(o));
-          acc[0] = fmaf(w, t.x, acc[0]);
-          acc[1] = fmaf(w, t.y, acc[1]);
-        }
-      }
-    }
-    const float inv = 1.0f / den;
-    const size_t o = (static_cast<size_t>(b) * a.q_heads + head0 + h) * D + lane * PER;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) store_out(a.out, a.out_dtype, o + i, acc[i] * inv);
-  }
-}
-
 template <class C>
 __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a) {
   constexpr int D = C::D, NG = C::NG, NQ = C::NQ, NP = C::NP, QS = C::QS, HT = C::HT;
@@ -297,7 +233,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   const int nh = min(a.heads_per_cta, a.gq - hg * a.heads_per_cta);
   if (t0 >= len) {
     // an empty sequence attends to nothing: its output rows are zero
-    if (a.fused && len == 0 && split == 0)
+    if (a.direct && len == 0 && split == 0)
       for (int i = threadIdx.x; i < nh * D; i += C::kThreads)
         store_out(a.out, a.out_dtype,
                   (static_cast<size_t>(b) * a.q_heads + head0 + i / D) * D + i % D, 0.0f);
@@ -808,9 +744,8 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   }
 
   // ------------------------------------------------------------ epilogue
-  // splits with tokens for this batch row; with one, this CTA's result is final
-  const int ns_b = (len + a.split_tokens - 1) / a.split_tokens;
-  const bool direct = a.fused && ns_b == 1;
+  // with one split per row this CTA's result is final
+  const bool direct = a.direct;
   __syncthreads();  // all stages consumed; the ring becomes the merge buffer
   float* ob = reinterpret_cast<float*>(smem);  // [warp][8][D]
   float* mb = mrg;                             // [warp][8]
@@ -886,25 +821,6 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     } else {
       const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * a.num_splits + split;
       a.ws_o[row * D + d] = num * rden[head];
-    }
-  }
-  if (a.fused && ns_b > 1) {
-    // publish this split, then the last CTA of the unit merges all of them
-    __threadfence();
-    __syncthreads();
-    int* s_last = reinterpret_cast<int*>(rden + 8);
-    if (threadIdx.x == 0) {
-      unsigned long long* ctr = a.counters + (static_cast<size_t>(b) * gridDim.y + blockIdx.y);
-      const bool last = arrive_last(ctr, a.epoch, ns_b, a.err);
-      *s_last = last;
-    }
-    __syncthreads();
-    if (*s_last) {
-      __threadfence();
-      merge_partials<D, C::kWarps>(a, b, head0, nh, ns_b);
-      if (threadIdx.x == 0)
-        a.counters[static_cast<size_t>(b) * gridDim.y + blockIdx.y] =
-            static_cast<unsigned long long>(a.epoch) << 32;
     }
   }
 }

@@ -64,14 +64,11 @@ struct DecodeArgs {
   float* ws_o;        // [B][Hq][num_splits][D] partial outputs
   float* ws_lse;      // [B][Hq][num_splits] log2-domain log-sum-exp
   uint32_t* err;
-  // Merge inside the kernel: a row with one split writes `out` directly; with
-  // more, the last CTA of each (batch row, kv head x head group) to arrive
-  // (counters[unit] = epoch << 32 | arrivals) merges the partials into `out`.
-  bool fused;
+  // One split per row (num_splits == 1): each CTA writes its rows' final
+  // output to `out` (no partials, no combine launch).
+  bool direct;
   void* out;
   int out_dtype;
-  unsigned long long* counters;
-  uint32_t epoch;
 };
 
 // Kernel variant, from the query type and the number of heads per CTA:
