@@ -77,6 +77,8 @@ def sha_of(paths):
 
 KERNEL_SOURCES = {
     "quantize": ["kv_cache_mixed_kvq_b200/csrc/quantize.cuh", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
+    "quantize_rot": ["kv_cache_mixed_kvq_b200/csrc/quantize.cuh",
+                     "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
     "decode": ["kv_cache_mixed_kvq_b200/csrc/decode.cuh", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
     "combine": ["kv_cache_mixed_kvq_b200/csrc/combine.cu", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
 }
@@ -295,7 +297,9 @@ def run_ours(args, rank, world, device):
         roof[name] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak,
                       "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
                       "traffic": measured_traffic(
-                          ["quantize"] if key == "quantize" else ["decode", "combine"], w.name),
+                          (["quantize_rot"] if args.rotate_keys else ["quantize"])
+                          if key == "quantize" else
+                          (["decode"] if arm.num_splits == 1 else ["decode", "combine"]), w.name),
                       "ms": round(kern[name], 5), "algorithmic_bytes": nbytes[key],
                       "peak_source": f"{peak_kind} hbm_gbs (copy)"}
     dominant = "quantize" if "quantize" in roof and kern["quantize"] >= kern.get(
