@@ -69,6 +69,11 @@ def _load(path: str | None = None):
     lib.ora_decode_attention_ex.argtypes = [I] * 7 + [P] * 4 + [P, I, I, P, I, ctypes.c_float,
                                                               I, P]
     lib.ora_decode_attention_ex.restype = I
+    lib.ora_quantize_append_g2.argtypes = [I] * 8 + [P] * 6 + [I, P, I, I]
+    lib.ora_quantize_append_g2.restype = I
+    lib.ora_decode_attention_g2.argtypes = [I] * 8 + [P] * 4 + [P, I, I, P, I, ctypes.c_float,
+                                                              I, P]
+    lib.ora_decode_attention_g2.restype = I
     return lib
 
 
@@ -140,16 +145,18 @@ def v_code_place(D: int, bits: int, k: int, d: int):
 class HostCache:
     """Host copies of the four cache arrays in the library's format."""
 
-    def __init__(self, B, Hkv, D, capacity, bits_k, bits_v, group, rotate_keys=False):
+    def __init__(self, B, Hkv, D, capacity, bits_k, bits_v, group, rotate_keys=False,
+                 group_v=None):
         self.B, self.Hkv, self.D, self.cap = B, Hkv, D, capacity
         self.bits_k, self.bits_v, self.group = bits_k, bits_v, group
+        self.group_v = group if not group_v else group_v  # values' group size
         self.rotate_keys = bool(rotate_keys)  # keys stored as H k (Walsh-Hadamard)
         slots = B * Hkv
         self.k_codes = np.zeros(slots * capacity * D * bits_k // 8, np.uint8)
         self.v_codes = np.zeros(slots * capacity * D * bits_v // 8, np.uint8)
         ng = D // group
         self.k_params = np.zeros(slots * capacity * ng * 2, np.uint16)
-        self.v_params = np.zeros(slots * capacity * ng * 2, np.uint16)
+        self.v_params = np.zeros(slots * capacity * (D // self.group_v) * 2, np.uint16)
 
     def _shape(self):
         return (self.B, self.Hkv, self.D, self.cap, self.bits_k, self.bits_v, self.group)
@@ -162,10 +169,10 @@ class HostCache:
         assert k.shape == (self.B, self.Hkv, n_new, self.D) and v.shape == k.shape
         pos = np.ascontiguousarray(pos, dtype=np.int32)
         dt = DTYPE_CODE[_dtype_of(k, dtype)]
-        r = lib().ora_quantize_append_ex(*self._shape(), _ptr(self.k_codes), _ptr(self.v_codes),
-                                         _ptr(self.k_params), _ptr(self.v_params),
-                                         _ptr(k), _ptr(v), dt, _ptr(pos), n_new,
-                                         int(self.rotate_keys))
+        r = lib().ora_quantize_append_g2(*self._shape(), self.group_v, _ptr(self.k_codes),
+                                         _ptr(self.v_codes), _ptr(self.k_params),
+                                         _ptr(self.v_params), _ptr(k), _ptr(v), dt, _ptr(pos),
+                                         n_new, int(self.rotate_keys))
         if r < 0:
             raise ValueError("invalid cache shape")
         return r
@@ -178,7 +185,8 @@ class HostCache:
 
     def dequant_row(self, which: int, b: int, h: int, p: int) -> np.ndarray:
         out = np.zeros(self.D, np.float32)
-        lib().ora_dequant_row(self.Hkv, self.D, self.cap, self.bits_k, self.bits_v, self.group,
+        lib().ora_dequant_row(self.Hkv, self.D, self.cap, self.bits_k, self.bits_v,
+                              self.group if which == 0 else self.group_v,
                               _ptr(self.k_codes), _ptr(self.v_codes), _ptr(self.k_params),
                               _ptr(self.v_params), which, b, h, p, _ptr(out))
         return out
@@ -194,7 +202,8 @@ class HostCache:
         assert q.shape == (self.B, Hq, self.D)
         lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
         out = np.zeros((self.B, Hq, self.D), np.float64)
-        r = lib().ora_decode_attention_ex(*self._shape(), _ptr(self.k_codes), _ptr(self.v_codes),
+        r = lib().ora_decode_attention_g2(*self._shape(), self.group_v, _ptr(self.k_codes),
+                                          _ptr(self.v_codes),
                                        _ptr(self.k_params), _ptr(self.v_params), _ptr(q),
                                        DTYPE_CODE[_dtype_of(q, q_dtype)], Hq, _ptr(lens),
                                        self.cap if max_len is None else max_len,

@@ -26,6 +26,11 @@
  *     dequantised cache (plain definition of one decode step of attention).
  *   - ora_attention_dense: the same on unquantised K/V (the full-precision
  *     baseline of "Results", "Downstream accuracy").
+ *   - separate group sizes (the *_g2 variants): "Results", "Group-size
+ *     sensitivity": finer groups (32) help the keys, coarser ones (64 or 128)
+ *     are enough for the values; keys use groups of Gk elements and values
+ *     groups of Gv, each array's (scale, zero) pairs indexed by its own
+ *     group count D/Gk or D/Gv.
  *   - ora_fwht and the *_ex variants: key-only rotation ("Results",
  *     "Integration with rotation": rotating only the keys in a K4V2 setting
  *     comes close to K4V4; the page names no transform, the plainest reading
@@ -223,13 +228,12 @@ static void fwht_d(double* x, int n) {
  * dtype, batch row b writes positions pos[b] .. pos[b]+n_new-1.  A batch row
  * whose range leaves [0, cap) is skipped.  Returns the flags: 1 = past
  * capacity, 8 = negative position; -1 for an invalid shape. */
-int ora_quantize_append_ex(int B, int Hkv, int D, int cap, int bk, int bv, int G,
+int ora_quantize_append_g2(int B, int Hkv, int D, int cap, int bk, int bv, int Gk, int Gv,
                            uint8_t* k_codes, uint8_t* v_codes, uint16_t* k_params,
                            uint16_t* v_params, const void* k, const void* v,
                            int dtype, const int32_t* pos, int n_new, int rotate_keys) {
-  if (!valid_shape(D, cap, bk, bv, G)) return -1;
+  if (!valid_shape(D, cap, bk, bv, Gk) || !valid_shape(D, cap, bk, bv, Gv)) return -1;
   int flags = 0;
-  int NG = D / G;
   size_t krow = (size_t)D * bk / 8;
   size_t vtile = (size_t)2 * D * bv;
   float* x = (float*)malloc(sizeof(float) * D);
@@ -251,6 +255,8 @@ int ora_quantize_append_ex(int B, int Hkv, int D, int cap, int bk, int bv, int G
         for (int which = 0; which < 2; ++which) {
           const void* in = which == 0 ? k : v;
           int bits = which == 0 ? bk : bv;
+          int G = which == 0 ? Gk : Gv;
+          int NG = D / G;
           uint16_t* params = which == 0 ? k_params : v_params;
           for (int d = 0; d < D; ++d) x[d] = load_elem(in, dtype, src + d);
           if (which == 0 && rotate_keys) ora_fwht(x, D);
@@ -284,6 +290,14 @@ int ora_quantize_append_ex(int B, int Hkv, int D, int cap, int bk, int bv, int G
   return flags;
 }
 
+int ora_quantize_append_ex(int B, int Hkv, int D, int cap, int bk, int bv, int G,
+                           uint8_t* k_codes, uint8_t* v_codes, uint16_t* k_params,
+                           uint16_t* v_params, const void* k, const void* v,
+                           int dtype, const int32_t* pos, int n_new, int rotate_keys) {
+  return ora_quantize_append_g2(B, Hkv, D, cap, bk, bv, G, G, k_codes, v_codes, k_params,
+                                v_params, k, v, dtype, pos, n_new, rotate_keys);
+}
+
 int ora_quantize_append(int B, int Hkv, int D, int cap, int bk, int bv, int G,
                         uint8_t* k_codes, uint8_t* v_codes, uint16_t* k_params,
                         uint16_t* v_params, const void* k, const void* v,
@@ -313,7 +327,8 @@ void ora_read_codes(int Hkv, int D, int cap, int bk, int bv, const uint8_t* k_co
   }
 }
 
-/* Dequantised row: x^_d = code_d * scale16 + zero16, in binary32. */
+/* Dequantised row: x^_d = code_d * scale16 + zero16, in binary32.  G is the
+ * group size of the array read (which = 0: keys, 1: values). */
 void ora_dequant_row(int Hkv, int D, int cap, int bk, int bv, int G,
                      const uint8_t* k_codes, const uint8_t* v_codes,
                      const uint16_t* k_params, const uint16_t* v_params,
@@ -361,13 +376,14 @@ static void attend(int D, int len, const double* q, const float* k_rows,
  * Batch row b attends to positions [0, min(seq_lens[b], max_len, cap)).
  * sm_scale <= 0 selects 1/sqrt(D).  Returns 2 if a length was clamped,
  * -1 on an invalid shape, else 0. */
-int ora_decode_attention_ex(int B, int Hkv, int D, int cap, int bk, int bv, int G,
+int ora_decode_attention_g2(int B, int Hkv, int D, int cap, int bk, int bv, int Gk, int Gv,
                             const uint8_t* k_codes, const uint8_t* v_codes,
                             const uint16_t* k_params, const uint16_t* v_params,
                             const void* q, int q_dtype, int Hq,
                             const int32_t* seq_lens, int max_len, float sm_scale,
                             int rotate_keys, double* out) {
-  if (!valid_shape(D, cap, bk, bv, G) || Hq % Hkv) return -1;
+  if (!valid_shape(D, cap, bk, bv, Gk) || !valid_shape(D, cap, bk, bv, Gv) || Hq % Hkv)
+    return -1;
   int flags = 0;
   int gq = Hq / Hkv;
   double scale = sm_scale > 0.0f ? (double)sm_scale : 1.0 / sqrt((double)D);
@@ -384,9 +400,9 @@ int ora_decode_attention_ex(int B, int Hkv, int D, int cap, int bk, int bv, int 
       float* kr = (float*)malloc(sizeof(float) * (size_t)(len > 0 ? len : 1) * D);
       float* vr = (float*)malloc(sizeof(float) * (size_t)(len > 0 ? len : 1) * D);
       for (int t = 0; t < len; ++t) {
-        ora_dequant_row(Hkv, D, cap, bk, bv, G, k_codes, v_codes, k_params, v_params,
+        ora_dequant_row(Hkv, D, cap, bk, bv, Gk, k_codes, v_codes, k_params, v_params,
                         0, b, h, t, kr + (size_t)t * D);
-        ora_dequant_row(Hkv, D, cap, bk, bv, G, k_codes, v_codes, k_params, v_params,
+        ora_dequant_row(Hkv, D, cap, bk, bv, Gv, k_codes, v_codes, k_params, v_params,
                         1, b, h, t, vr + (size_t)t * D);
       }
       for (int j = 0; j < gq; ++j) {
@@ -406,6 +422,17 @@ int ora_decode_attention_ex(int B, int Hkv, int D, int cap, int bk, int bv, int 
   }
   free(qd);
   return flags;
+}
+
+int ora_decode_attention_ex(int B, int Hkv, int D, int cap, int bk, int bv, int G,
+                            const uint8_t* k_codes, const uint8_t* v_codes,
+                            const uint16_t* k_params, const uint16_t* v_params,
+                            const void* q, int q_dtype, int Hq,
+                            const int32_t* seq_lens, int max_len, float sm_scale,
+                            int rotate_keys, double* out) {
+  return ora_decode_attention_g2(B, Hkv, D, cap, bk, bv, G, G, k_codes, v_codes, k_params,
+                                 v_params, q, q_dtype, Hq, seq_lens, max_len, sm_scale,
+                                 rotate_keys, out);
 }
 
 int ora_decode_attention(int B, int Hkv, int D, int cap, int bk, int bv, int G,

@@ -16,6 +16,7 @@ from tests import test_oracle_layout as lay
 from tests import test_oracle_numbers as num
 from tests import test_oracle_quantizer as qz
 from tests import test_oracle_rotation as rot
+from tests import test_oracle_groups as grp
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "kvq_oracle.c")
 
@@ -43,6 +44,10 @@ MUTANTS = {
     "keys_not_rotated": ("if (which == 0 && rotate_keys) ora_fwht(x, D);", ""),
     "values_rotated_too": ("if (which == 0 && rotate_keys) ora_fwht(x, D);",
                            "if (rotate_keys) ora_fwht(x, D);"),
+    # separate key and value groups
+    # (keys quantized with the values' coarser groups; writes stay inside the
+    # key-parameter array, which is sized for the finer groups)
+    "key_groups_from_values": ("int G = which == 0 ? Gk : Gv;", "int G = Gv;"),
 }
 
 PINS = [
@@ -64,6 +69,7 @@ PINS = [
     lambda o: rot.test_fwht_is_the_sylvester_hadamard_product(o, 64),
     lambda o: rot.test_rotated_keys_dequantise_near_the_rotated_row(o),
     lambda o: rot.test_rotated_decode_matches_dense_attention_at_8_bits(o),
+    lambda o: grp.test_each_array_uses_its_own_groups(o, 32, 128),
 ]
 
 
