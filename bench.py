@@ -54,12 +54,13 @@ def step_shape(w: workloads.Workload, bits):
     return n_new, pos, read
 
 
-def algorithmic_bytes(w: workloads.Workload, bits, n_new, read_lens):
+def algorithmic_bytes(w: workloads.Workload, bits, n_new, read_lens, group_v: int = 0):
     """HBM bytes the step must move, by kernel (what the method reads/writes)."""
     bk, bv = bits
     D, G = w.head_dim, w.group
+    Gv = group_v or G
     el = 4 if w.dtype == "f32" else 2
-    per_tok_cache = D * (bk + bv) // 8 + 2 * (D // G) * 4
+    per_tok_cache = D * (bk + bv) // 8 + (D // G) * 4 + (D // Gv) * 4
     rows = w.batch * w.kv_heads * n_new
     quant = rows * (2 * D * el + per_tok_cache) + 4 * w.batch
     tokens = sum(read_lens)
@@ -174,7 +175,8 @@ class ClockSampler:
 class Arm:
     """Device buffers for R rotating sets of inputs + caches, and the step."""
 
-    def __init__(self, w, bits, rotate: int, device, rotate_keys: bool = False):
+    def __init__(self, w, bits, rotate: int, device, rotate_keys: bool = False,
+                 group_v: int = 0):
         import kv_cache_mixed_kvq_b200 as kvq
         self.kvq = kvq
         self.w, self.bits = w, bits
@@ -187,7 +189,7 @@ class Arm:
         for r in range(rotate):
             cache = kvq.KVCache.allocate(w.batch, w.kv_heads, w.head_dim, self.cap, bits[0],
                                          bits[1], w.group, device=device,
-                                         rotate_keys=rotate_keys)
+                                         rotate_keys=rotate_keys, group_v=group_v)
             if w.name != "llama3_8b":
                 # pre-fill the context (untimed); the step then appends n_new tokens
                 for b in range(w.batch):
@@ -232,7 +234,7 @@ def _slot_view(cache, b):
                        cache.bits_v, cache.group,
                        *[t[b * n:(b + 1) * n] for t, n in zip(
                            (cache.k_codes, cache.v_codes, cache.k_params, cache.v_params), per)],
-                       rotate_keys=cache.rotate_keys)
+                       rotate_keys=cache.rotate_keys, group_v=cache.group_v)
 
 
 def run_ours(args, rank, world, device):
@@ -240,7 +242,7 @@ def run_ours(args, rank, world, device):
     bits = tuple(int(x) for x in args.bits.split(",")) if args.bits else w.bits[-1] \
         if w.name == "long" else w.bits[0]
     rotate = args.rotate
-    arm = Arm(w, bits, rotate, device, rotate_keys=args.rotate_keys)
+    arm = Arm(w, bits, rotate, device, rotate_keys=args.rotate_keys, group_v=args.group_v)
     stream = torch.cuda.current_stream()
 
     # warm-up (also loads every kernel and the error-word address)
@@ -282,7 +284,7 @@ def run_ours(args, rank, world, device):
     ms_step = ms / args.steps
     flags = arm.kvq.kvq_device_error_flags()
 
-    nbytes = algorithmic_bytes(w, bits, arm.n_new, arm.read)
+    nbytes = algorithmic_bytes(w, bits, arm.n_new, arm.read, args.group_v)
     step_bytes = nbytes["quantize"] * (1 if arm.n_new else 0) + nbytes["decode"]
 
     # ---------------- per-kernel durations (events inside a graph, GPU kept busy)
@@ -325,6 +327,7 @@ def run_ours(args, rank, world, device):
             "head_dim": w.head_dim, "context": w.context, "input_dtype": w.dtype,
             "bits_k": bits[0], "bits_v": bits[1], "group": w.group,
             "rotate_keys": bool(args.rotate_keys),
+            "group_v": args.group_v or w.group,
             "step": ("quantize full cache + decode + combine" if w.name == "llama3_8b" else
                      f"append {arm.n_new} + decode + combine"),
             "split_tokens": arm.split_tokens,
@@ -525,6 +528,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--group-v", type=int, default=0,
+                    help="values' group size (default: the workload's group)")
     ap.add_argument("--rotate-keys", action="store_true",
                     help="cache with key-only Walsh-Hadamard rotation (KVQ_FLAG_ROTATE_KEYS)")
     args = ap.parse_args()

@@ -50,10 +50,11 @@
  *
  *   k_codes : capacity * (D * b_k / 8) bytes per slot  (K rows)
  *   v_codes : capacity * (D * b_v / 8) bytes per slot  (V tiles)
- *   k_params: capacity * (D / G) * 4   bytes per slot  (K scale/zero)
- *   v_params: capacity * (D / G) * 4   bytes per slot  (V scale/zero)
+ *   k_params: capacity * (D / Gk) * 4  bytes per slot  (K scale/zero)
+ *   v_params: capacity * (D / Gv) * 4  bytes per slot  (V scale/zero)
  *
- * Params: for token position p and group g, the 4 bytes at offset
+ * Gk = group, Gv = group_v (or group).  Params: for token position p and
+ * group g of an array with group size G, the 4 bytes at offset
  * (p * (D/G) + g) * 4 hold binary16 scale (lower address) then binary16 zero.
  *
  * K rows (token-major; row p at byte offset p * D*b/8 of the slot).  With
@@ -156,7 +157,10 @@ enum kvq_cache_array {
  *   capacity >= 16 and a multiple of 16 token positions per slot,
  *   bits_k, bits_v in {2, 4, 8} (the page's key-priority rule is b_k > b_v;
  *   other orders are accepted so that they can be compared),
- *   group (G) in {32, 64, 128} with G <= D.
+ *   group (G) in {32, 64, 128} with G <= D: the keys' group size;
+ *   group_v: the values' group size, 0 (= group) or in {32, 64, 128} with
+ *   group <= group_v <= D ("Results", "Group-size sensitivity": finer
+ *   groups help the keys, coarser ones are enough for the values).
  * Pointers: device memory, 16-byte aligned, sized by kvq_cache_bytes().
  */
 typedef struct kvq_cache_desc {
@@ -168,6 +172,8 @@ typedef struct kvq_cache_desc {
   int32_t bits_v;
   int32_t group;
   int32_t flags;    /* kvq_cache_flags; other bits must be 0 */
+  int32_t group_v;  /* values' group size; 0: same as group */
+  int32_t reserved; /* must be 0 */
   uint8_t* k_codes;
   uint8_t* v_codes;
   void* k_params; /* binary16 (scale, zero) pairs */
@@ -176,7 +182,8 @@ typedef struct kvq_cache_desc {
 
 /*
  * Bytes of one cache array for the given shape (all slots), or 0 if the
- * shape is invalid.  Pure host function.
+ * shape is invalid.  `group` is the group size of the array asked for: the
+ * keys' for KVQ_K_PARAMS, the values' for KVQ_V_PARAMS.  Pure host function.
  */
 size_t kvq_cache_bytes(int32_t batch, int32_t kv_heads, int32_t head_dim,
                        int32_t capacity, int32_t bits_k, int32_t bits_v,

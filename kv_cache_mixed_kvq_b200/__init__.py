@@ -46,6 +46,7 @@ class KvqCacheDesc(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("capacity", ctypes.c_int32),
         ("bits_k", ctypes.c_int32), ("bits_v", ctypes.c_int32),
         ("group", ctypes.c_int32), ("flags", ctypes.c_int32),
+        ("group_v", ctypes.c_int32), ("reserved", ctypes.c_int32),
         ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
         ("k_params", ctypes.c_void_p), ("v_params", ctypes.c_void_p),
     ]
@@ -130,22 +131,24 @@ class KVCache:
     k_params: torch.Tensor
     v_params: torch.Tensor
     rotate_keys: bool = False  # KVQ_FLAG_ROTATE_KEYS: keys stored as H k
+    group_v: int = 0           # values' group size (0: same as group)
 
     @classmethod
     def allocate(cls, batch, kv_heads, head_dim, capacity, bits_k, bits_v, group,
-                 device="cuda", rotate_keys: bool = False) -> "KVCache":
-        sizes = [kvq_cache_bytes(batch, kv_heads, head_dim, capacity, bits_k, bits_v, group, w)
-                 for w in range(4)]
+                 device="cuda", rotate_keys: bool = False, group_v: int = 0) -> "KVCache":
+        gv = group_v or group
+        sizes = [kvq_cache_bytes(batch, kv_heads, head_dim, capacity, bits_k, bits_v,
+                                 gv if w == KVQ_V_PARAMS else group, w) for w in range(4)]
         if 0 in sizes:
             raise KvqError(KVQ_ERR_INVALID_ARG, "KVCache.allocate")
         bufs = [torch.zeros(n, dtype=torch.uint8, device=device) for n in sizes]
         return cls(batch, kv_heads, head_dim, capacity, bits_k, bits_v, group, *bufs,
-                   rotate_keys=rotate_keys)
+                   rotate_keys=rotate_keys, group_v=group_v)
 
     def desc(self) -> KvqCacheDesc:
         return KvqCacheDesc(self.batch, self.kv_heads, self.head_dim, self.capacity,
                             self.bits_k, self.bits_v, self.group,
-                            KVQ_FLAG_ROTATE_KEYS if self.rotate_keys else 0,
+                            KVQ_FLAG_ROTATE_KEYS if self.rotate_keys else 0, self.group_v, 0,
                             _dev_ptr(self.k_codes, "k_codes"), _dev_ptr(self.v_codes, "v_codes"),
                             _dev_ptr(self.k_params, "k_params"), _dev_ptr(self.v_params, "v_params"))
 

@@ -13,19 +13,19 @@
 #include "internal.h"
 
 namespace kvq {
-bool get_decode_kernel_k2v2(int, int, int, DecodeKernel*);
-bool get_decode_kernel_k2v4(int, int, int, DecodeKernel*);
-bool get_decode_kernel_k2v8(int, int, int, DecodeKernel*);
-bool get_decode_kernel_k4v2(int, int, int, DecodeKernel*);
-bool get_decode_kernel_k4v4(int, int, int, DecodeKernel*);
-bool get_decode_kernel_k4v8(int, int, int, DecodeKernel*);
-bool get_decode_kernel_k8v2(int, int, int, DecodeKernel*);
-bool get_decode_kernel_k8v4(int, int, int, DecodeKernel*);
-bool get_decode_kernel_k8v8(int, int, int, DecodeKernel*);
+bool get_decode_kernel_k2v2(int, int, int, int, DecodeKernel*);
+bool get_decode_kernel_k2v4(int, int, int, int, DecodeKernel*);
+bool get_decode_kernel_k2v8(int, int, int, int, DecodeKernel*);
+bool get_decode_kernel_k4v2(int, int, int, int, DecodeKernel*);
+bool get_decode_kernel_k4v4(int, int, int, int, DecodeKernel*);
+bool get_decode_kernel_k4v8(int, int, int, int, DecodeKernel*);
+bool get_decode_kernel_k8v2(int, int, int, int, DecodeKernel*);
+bool get_decode_kernel_k8v4(int, int, int, int, DecodeKernel*);
+bool get_decode_kernel_k8v8(int, int, int, int, DecodeKernel*);
 
-bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int num_groups, int variant,
-                       DecodeKernel* out) {
-  using Fn = bool (*)(int, int, int, DecodeKernel*);
+bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int groups_k, int groups_v,
+                       int variant, DecodeKernel* out) {
+  using Fn = bool (*)(int, int, int, int, DecodeKernel*);
   static const Fn table[3][3] = {
       {get_decode_kernel_k2v2, get_decode_kernel_k2v4, get_decode_kernel_k2v8},
       {get_decode_kernel_k4v2, get_decode_kernel_k4v4, get_decode_kernel_k4v8},
@@ -33,7 +33,7 @@ bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int num_groups, int
   auto idx = [](int b) { return b == 2 ? 0 : b == 4 ? 1 : b == 8 ? 2 : -1; };
   const int i = idx(bits_k), j = idx(bits_v);
   if (i < 0 || j < 0) return false;
-  return table[i][j](head_dim, num_groups, variant, out);
+  return table[i][j](head_dim, groups_k, groups_v, variant, out);
 }
 }  // namespace kvq
 
@@ -62,11 +62,20 @@ int check_shape(int B, int Hkv, int D, int cap, int bk, int bv, int G) {
   return KVQ_OK;
 }
 
+// Values' group size (group_v = 0 means the keys' group).
+int group_v_of(const kvq_cache_desc* c) { return c->group_v != 0 ? c->group_v : c->group; }
+
 int check_cache(const kvq_cache_desc* c) {
-  if (!c || (c->flags & ~KVQ_FLAG_ROTATE_KEYS) != 0) return KVQ_ERR_INVALID_ARG;
-  const int st = check_shape(c->batch, c->kv_heads, c->head_dim, c->capacity, c->bits_k,
-                             c->bits_v, c->group);
+  if (!c || (c->flags & ~KVQ_FLAG_ROTATE_KEYS) != 0 || c->reserved != 0)
+    return KVQ_ERR_INVALID_ARG;
+  int st = check_shape(c->batch, c->kv_heads, c->head_dim, c->capacity, c->bits_k, c->bits_v,
+                       c->group);
   if (st != KVQ_OK) return st;
+  const int gv = group_v_of(c);
+  st = check_shape(c->batch, c->kv_heads, c->head_dim, c->capacity, c->bits_k, c->bits_v, gv);
+  if (st != KVQ_OK) return st;
+  // instances exist for equal groups and for coarser value groups
+  if (gv < c->group) return KVQ_ERR_UNSUPPORTED;
   const void* ptrs[4] = {c->k_codes, c->v_codes, c->k_params, c->v_params};
   for (const void* p : ptrs)
     if (!p || !aligned(p, 16)) return KVQ_ERR_INVALID_ARG;
@@ -142,6 +151,7 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
   }
   DecodeKernel k;
   if (!kvq::get_decode_kernel(c->head_dim, c->bits_k, c->bits_v, c->head_dim / c->group,
+                              c->head_dim / group_v_of(c),
                               variant_of(p->heads_per_cta, KVQ_BF16), &k))
     return KVQ_ERR_UNSUPPORTED;
   int dev = 0, sms = 0, per_sm = 0;
@@ -265,6 +275,7 @@ int kvq_quantize_append(const kvq_cache_desc* cache, const void* k, const void* 
   a.bits_k = cache->bits_k;
   a.bits_v = cache->bits_v;
   a.group = cache->group;
+  a.group_v = group_v_of(cache);
   a.rotate_keys = (cache->flags & KVQ_FLAG_ROTATE_KEYS) != 0;
   st = error_word(&a.err);
   if (st != KVQ_OK) return st;
@@ -310,6 +321,7 @@ int kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int32_t q_d
   if (p.num_splits > 0) {
     DecodeKernel k;
     if (!kvq::get_decode_kernel(D, cache->bits_k, cache->bits_v, D / cache->group,
+                                D / group_v_of(cache),
                                 variant_of(p.heads_per_cta, q_dtype), &k))
       return KVQ_ERR_UNSUPPORTED;
     if (prepare_kernel(k) != cudaSuccess) return KVQ_ERR_CUDA;

@@ -36,14 +36,16 @@ namespace kvq {
 
 // QS == 2: each lane's two score columns are the high and low parts of one
 // head (up to 4 heads per n-tile); QS == 1: two heads (up to 8 per n-tile).
-template <int D_, int BK_, int BV_, int NG_, int QS_, int NQ_, int NP_>
+// NGK / NGV: groups per row of the keys / values (separate group sizes).
+template <int D_, int BK_, int BV_, int NGK_, int NGV_, int QS_, int NQ_, int NP_>
 struct DecodeCfg {
-  static constexpr int D = D_, BK = BK_, BV = BV_, NG = NG_, QS = QS_, NQ = NQ_, NP = NP_;
+  static constexpr int D = D_, BK = BK_, BV = BV_, QS = QS_, NQ = NQ_, NP = NP_;
+  static constexpr int NGK = NGK_, NGV = NGV_;
   static constexpr int kWarps = 4;  // warps per CTA; each runs its own copy pipeline
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int TPW = 2;     // 16-token tiles per warp per stage
   static constexpr int kStageTokens = 16 * TPW * kWarps;
-  static constexpr int G = D / NG;
+  static constexpr int GK = D / NGK, GV = D / NGV;
   static constexpr int KSTEPS = D / 16;  // k-steps (scores) == m-tiles (output)
   static constexpr int KROW = D * BK / 8;
   static constexpr int KSLICE = D * BK / 32;  // bytes of one lane's K slice
@@ -53,12 +55,12 @@ struct DecodeCfg {
   static constexpr int VP = VN < 16 ? VN : 16;
   static constexpr int VW = VN / 4;
   static constexpr int WV = D * BV / 128;  // V words per half-lane
-  static constexpr int PROW = NG * 4;
+  static constexpr int PROWK = NGK * 4, PROWV = NGV * 4;  // parameter bytes per position
   // one slot = one warp's 16*TPW positions of a stage: K rows, V tiles, K params, V params
   static constexpr int SLOT_K = 16 * TPW * KROW;
   static constexpr int SLOT_V = TPW * VTILE;
-  static constexpr int SLOT_P = 16 * TPW * PROW;
-  static constexpr int SLOT_BYTES = SLOT_K + SLOT_V + 2 * SLOT_P;
+  static constexpr int SLOT_PK = 16 * TPW * PROWK, SLOT_PV = 16 * TPW * PROWV;
+  static constexpr int SLOT_BYTES = SLOT_K + SLOT_V + SLOT_PK + SLOT_PV;
   // Copies in flight per warp.  Two slots measured as fast as three or four
   // on every workload shape (graph replay on B200), with a third less
   // shared memory.
@@ -66,17 +68,18 @@ struct DecodeCfg {
   static constexpr int RING_BYTES = kWarps * kSlots * SLOT_BYTES;
   // staged output weights: per warp and tile [group][head][part][WB_RS halves]
   static constexpr int WB_RS = 24;  // halves per row: 16 positions + pad (conflict-free)
-  static constexpr int WB_HALVES = NG * 8 * 2 * WB_RS;
+  static constexpr int WB_HALVES = NGV * 8 * 2 * WB_RS;
   static constexpr int WB_BYTES = TPW * kWarps * WB_HALVES * 2;
   static constexpr int ALPHA_FLOATS = kWarps * 8;
-  static constexpr int MERGE_FLOATS = kWarps * 8 * (2 + NG) + 2 * 8 * (kWarps + 1);
+  static constexpr int MERGE_FLOATS = kWarps * 8 * (2 + NGV) + 2 * 8 * (kWarps + 1);
   static constexpr int SMEM_BYTES =
       RING_BYTES + WB_BYTES + 4 * (ALPHA_FLOATS + MERGE_FLOATS) + 8 * kWarps * kSlots;
   static constexpr int HT = QS == 1 ? 2 * NQ : NQ;  // score head slots per lane
   static_assert(RING_BYTES >= kWarps * 8 * D * 4, "merge buffer must fit in the ring");
   static_assert(WB_BYTES >= 8 * D * 4, "rotated queries must fit in the staging buffer");
   static_assert(SLOT_BYTES % 16 == 0 && SLOT_K % 16 == 0 && SLOT_V % 16 == 0, "alignment");
-  static_assert(G >= 16 && G % 16 == 0, "group must cover whole 16-element steps");
+  static_assert(GK >= 16 && GK % 16 == 0 && GV >= 16 && GV % 16 == 0,
+                "groups must cover whole 16-element steps");
 };
 
 // Bit position and pre-shift of extraction e for b-bit fields: fields that
@@ -200,8 +203,8 @@ __device__ __forceinline__ void store_out(void* out, int dtype, size_t i, float 
 
 template <class C>
 __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a) {
-  constexpr int D = C::D, NG = C::NG, NQ = C::NQ, NP = C::NP, QS = C::QS, HT = C::HT;
-  constexpr int KSTEPS = C::KSTEPS, G = C::G;
+  constexpr int D = C::D, NGK = C::NGK, NGV = C::NGV, NQ = C::NQ, NP = C::NP, QS = C::QS;
+  constexpr int HT = C::HT, KSTEPS = C::KSTEPS, GK = C::GK, GV = C::GV;
   extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* wbuf = reinterpret_cast<uint16_t*>(smem + C::RING_BYTES);  // staged weights
   float* alph = reinterpret_cast<float*>(smem + C::RING_BYTES + C::WB_BYTES);  // [warp][8]
@@ -250,21 +253,22 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   uint8_t* wring = smem + warp * C::kSlots * C::SLOT_BYTES;
   const uint8_t* kb = a.k_codes + slot * a.capacity * C::KROW;
   const uint8_t* vb = a.v_codes + slot * (a.capacity / 16) * C::VTILE;
-  const uint8_t* kpb = reinterpret_cast<const uint8_t*>(a.k_params) + slot * a.capacity * C::PROW;
-  const uint8_t* vpb = reinterpret_cast<const uint8_t*>(a.v_params) + slot * a.capacity * C::PROW;
+  const uint8_t* kpb = reinterpret_cast<const uint8_t*>(a.k_params) + slot * a.capacity * C::PROWK;
+  const uint8_t* vpb = reinterpret_cast<const uint8_t*>(a.v_params) + slot * a.capacity * C::PROWV;
   auto issue = [&](int it, int sl) {
     const int base = it * C::kStageTokens + my_first;  // multiple of 16
     const int n16 = (min(16 * C::TPW, n_tok - base) + 15) & ~15;
     const int tb = t0 + base;
     uint8_t* dst = wring + sl * C::SLOT_BYTES;
-    const uint32_t kbytes = n16 * C::KROW, vbytes = (n16 / 16) * C::VTILE, pbytes = n16 * C::PROW;
-    mbar_arrive_expect_tx(&wfull[sl], kbytes + vbytes + 2 * pbytes);
+    const uint32_t kbytes = n16 * C::KROW, vbytes = (n16 / 16) * C::VTILE;
+    const uint32_t pkbytes = n16 * C::PROWK, pvbytes = n16 * C::PROWV;
+    mbar_arrive_expect_tx(&wfull[sl], kbytes + vbytes + pkbytes + pvbytes);
     bulk_copy_g2s(dst, kb + static_cast<size_t>(tb) * C::KROW, kbytes, &wfull[sl]);
     bulk_copy_g2s(dst + C::SLOT_K, vb + static_cast<size_t>(tb / 16) * C::VTILE, vbytes, &wfull[sl]);
-    bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V, kpb + static_cast<size_t>(tb) * C::PROW, pbytes,
+    bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V, kpb + static_cast<size_t>(tb) * C::PROWK, pkbytes,
                   &wfull[sl]);
-    bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V + C::SLOT_P, vpb + static_cast<size_t>(tb) * C::PROW,
-                  pbytes, &wfull[sl]);
+    bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V + C::SLOT_PK,
+                  vpb + static_cast<size_t>(tb) * C::PROWV, pvbytes, &wfull[sl]);
   };
   if (lane == 0)
     for (int it = 0; it < min(C::kSlots, my_iters); ++it) issue(it, it);
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   const int g = lane >> 2, c = lane & 3;
   float m_run[HT], l_run[HT];
   float oacc[KSTEPS][NP][4];
-  float2 zacc[HT][NG];  // zero term, score layout: (row g, row g+8) partials
+  float2 zacc[HT][NGV];  // zero term, score layout: (row g, row g+8) partials
   // Power-of-two exponent applied to the output weights p * scale_v so that
   // their binary16 parts stay normal; only ever decreases (see below).
   int u_run = 100;
@@ -293,7 +297,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
 #pragma unroll
   for (int hs = 0; hs < HT; ++hs)
 #pragma unroll
-    for (int gr = 0; gr < NG; ++gr) zacc[hs][gr] = make_float2(0.0f, 0.0f);
+    for (int gr = 0; gr < NGV; ++gr) zacc[hs][gr] = make_float2(0.0f, 0.0f);
 
   {
     // -------- query fragments (B operand of the score product), once per CTA
@@ -378,24 +382,24 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     // qz[gr][nt] = {col 2c, col 2c+1}; for QS == 2 both columns of a lane
     // belong to one head and are summed.
     const float F = a.sm_scale_log2 * pow2i(24 - eq);
-    float2 qz[NG][NQ];
+    float2 qz[NGK][NQ];
     {
-      float qsum[NG][NQ][4];
+      float qsum[NGK][NQ][4];
 #pragma unroll
       for (int j = 0; j < KSTEPS; ++j) {
-        const int gr = 16 * j / G;
+        const int gr = 16 * j / GK;
         const uint32_t one0 = 0x00010001u << field_pos<C::BK>((2 * j) % (16 / C::BK));
         const uint32_t one1 = 0x00010001u << field_pos<C::BK>((2 * j + 1) % (16 / C::BK));
 #pragma unroll
         for (int nt = 0; nt < NQ; ++nt) {
-          if (j % (G / 16) == 0)
+          if (j % (GK / 16) == 0)
             mma_f16_16816_zc(qsum[gr][nt], one0, one0, one1, one1, bq[nt][j][0], bq[nt][j][1]);
           else
             mma_f16_16816(qsum[gr][nt], one0, one0, one1, one1, bq[nt][j][0], bq[nt][j][1]);
         }
       }
 #pragma unroll
-      for (int gr = 0; gr < NG; ++gr)
+      for (int gr = 0; gr < NGK; ++gr)
 #pragma unroll
         for (int nt = 0; nt < NQ; ++nt)
           qz[gr][nt] = QS == 2 ? make_float2((qsum[gr][nt][0] + qsum[gr][nt][1]) * F, 0.0f)
@@ -414,7 +418,8 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     // lane offsets inside a stage (tile tt of this warp adds tt * 16 rows)
     const int k_off = g * C::KROW + c * C::KSLICE;
     const int v_off = C::SLOT_K + lane * C::VP;
-    const int kp_off = C::SLOT_K + C::SLOT_V + g * C::PROW;
+    const int kp_off = C::SLOT_K + C::SLOT_V + g * C::PROWK;
+    const int vp_off = C::SLOT_K + C::SLOT_V + C::SLOT_PK + g * C::PROWV;
     uint32_t* const err = a.err;
 
     // Process NTL consecutive tiles of this warp (tile indices t_first ..),
@@ -424,24 +429,25 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       constexpr bool FULL = decltype(full_tag)::value;
       constexpr int NTL = decltype(ntl_tag)::value;
       uint32_t kw[NTL][2 * C::KW];
-      uint32_t kpa[NTL][NG], kpb[NTL][NG], vpa[NTL][NG], vpb[NTL][NG];
+      uint32_t kpa[NTL][NGK], kpb[NTL][NGK], vpa[NTL][NGV], vpb[NTL][NGV];
 #pragma unroll
       for (int tt = 0; tt < NTL; ++tt) {
         const int tix = t_first + tt;
         lds_words<C::KSLICE>(st + k_off + tix * 16 * C::KROW, kw[tt], 0);
         lds_words<C::KSLICE>(st + k_off + (tix * 16 + 8) * C::KROW, kw[tt], C::KW);
         // (scale, zero) words of rows g and g+8: one vector load per row
-        const uint8_t* kp = st + kp_off + tix * 16 * C::PROW;
-        lds_words<C::PROW>(kp, kpa[tt], 0);
-        lds_words<C::PROW>(kp + 8 * C::PROW, kpb[tt], 0);
-        lds_words<C::PROW>(kp + C::SLOT_P, vpa[tt], 0);
-        lds_words<C::PROW>(kp + C::SLOT_P + 8 * C::PROW, vpb[tt], 0);
+        const uint8_t* kp = st + kp_off + tix * 16 * C::PROWK;
+        const uint8_t* vp = st + vp_off + tix * 16 * C::PROWV;
+        lds_words<C::PROWK>(kp, kpa[tt], 0);
+        lds_words<C::PROWK>(kp + 8 * C::PROWK, kpb[tt], 0);
+        lds_words<C::PROWV>(vp, vpa[tt], 0);
+        lds_words<C::PROWV>(vp + 8 * C::PROWV, vpb[tt], 0);
       }
       // ---- scores: S^T[token][col] = codes . q'
-      float acc[NTL][NG][NQ][4];
+      float acc[NTL][NGK][NQ][4];
 #pragma unroll
       for (int j = 0; j < KSTEPS; ++j) {
-        const int gr = 16 * j / G;
+        const int gr = 16 * j / GK;
 #pragma unroll
         for (int tt = 0; tt < NTL; ++tt) {
           const uint32_t a0 = extract_codes<C::BK>(kw[tt], 0, 2 * j);
@@ -450,7 +456,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
           const uint32_t a3 = extract_codes<C::BK>(kw[tt], C::KW, 2 * j + 1);
 #pragma unroll
           for (int nt = 0; nt < NQ; ++nt) {
-            if (j % (G / 16) == 0)
+            if (j % (GK / 16) == 0)
               mma_f16_16816_zc(acc[tt][gr][nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
             else
               mma_f16_16816(acc[tt][gr][nt], a0, a1, a2, a3, bq[nt][j][0], bq[nt][j][1]);
@@ -466,7 +472,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
           for (int nt = 0; nt < NQ; ++nt) {
             float2 t = make_float2(0.0f, 0.0f), z = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int gr = 0; gr < NG; ++gr) {
+            for (int gr = 0; gr < NGK; ++gr) {
               // rows (g, g+8): high + low columns
               const float2 sum = __fadd2_rn(make_float2(acc[tt][gr][nt][0], acc[tt][gr][nt][2]),
                                             make_float2(acc[tt][gr][nt][1], acc[tt][gr][nt][3]));
@@ -485,7 +491,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
             for (int nt = 0; nt < NQ; ++nt) {
               float2 t = make_float2(0.0f, 0.0f), z = make_float2(0.0f, 0.0f);
 #pragma unroll
-              for (int gr = 0; gr < NG; ++gr) {
+              for (int gr = 0; gr < NGK; ++gr) {
                 const float2 sz = unpack_half2(rr ? kpb[tt][gr] : kpa[tt][gr]);
                 t = __ffma2_rn(make_float2(sz.x, sz.x),
                                make_float2(acc[tt][gr][nt][2 * rr], acc[tt][gr][nt][2 * rr + 1]), t);
@@ -506,7 +512,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
           if (g + 8 >= nvalid) lg[0][hs][1] = -INFINITY;
         }
 #pragma unroll
-        for (int gr = 0; gr < NG; ++gr) {
+        for (int gr = 0; gr < NGV; ++gr) {
           if (g >= nvalid) vpa[0][gr] = 0u;
           if (g + 8 >= nvalid) vpb[0][gr] = 0u;
         }
@@ -533,7 +539,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
           const float alpha = mnew == -INFINITY ? 1.0f : exp2_approx(m_run[hs] - mnew);
           l_run[hs] *= alpha;
 #pragma unroll
-          for (int gr = 0; gr < NG; ++gr)
+          for (int gr = 0; gr < NGV; ++gr)
             zacc[hs][gr] = __fmul2_rn(zacc[hs][gr], make_float2(alpha, alpha));
           m_run[hs] = mnew;
           if (g == 0) walph[head] = alpha;
@@ -555,7 +561,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
 #pragma unroll
         for (int tt = 0; tt < NTL; ++tt)
 #pragma unroll
-          for (int gr = 0; gr < NG; ++gr) {
+          for (int gr = 0; gr < NGV; ++gr) {
             __half2 r = __hmax2(*reinterpret_cast<__half2*>(&hm), *reinterpret_cast<__half2*>(&vpa[tt][gr]));
             r = __hmax2(r, *reinterpret_cast<__half2*>(&vpb[tt][gr]));
             hm = *reinterpret_cast<uint32_t*>(&r);
@@ -586,9 +592,9 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         const float fu = pow2i(u_run);
 #pragma unroll
         for (int tt = 0; tt < NTL; ++tt) {
-          uint32_t mr[2 * NG * NP];
+          uint32_t mr[2 * NGV * NP];
 #pragma unroll
-          for (int gr = 0; gr < NG; ++gr) {
+          for (int gr = 0; gr < NGV; ++gr) {
             const float2 sc = scales_of(vpa[tt][gr], vpb[tt][gr]);
             const float2 zr = zeros_of(vpa[tt][gr], vpb[tt][gr]);
 #pragma unroll
@@ -597,15 +603,15 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
               const uint32_t hi = f2_to_h2(P.x, P.y);
               const float2 hf = unpack_half2(hi);
               const uint32_t lo = f2_to_h2(P.x - hf.x, P.y - hf.y);
-              mr[2 * (hs * NG + gr)] = __byte_perm(hi, lo, 0x5410);      // row g: (high, low)
-              mr[2 * (hs * NG + gr) + 1] = __byte_perm(hi, lo, 0x7632);  // row g + 8
+              mr[2 * (hs * NGV + gr)] = __byte_perm(hi, lo, 0x5410);      // row g: (high, low)
+              mr[2 * (hs * NGV + gr) + 1] = __byte_perm(hi, lo, 0x7632);  // row g + 8
               zacc[hs][gr] = __ffma2_rn(pr[tt][hs], zr, zacc[hs][gr]);
             }
           }
           uint8_t* wbt = reinterpret_cast<uint8_t*>(wb + (t_first + tt) * C::WB_HALVES);
 #pragma unroll
-          for (int m0 = 0; m0 < 2 * NG * NP; m0 += 4) {
-            if constexpr (2 * NG * NP >= 4)
+          for (int m0 = 0; m0 < 2 * NGV * NP; m0 += 4) {
+            if constexpr (2 * NGV * NP >= 4)
               stmatrix_b16<4>(wbt + m0 * 128 + lane * 16, mr + m0);
             else
               stmatrix_b16<2>(wbt + m0 * 128 + lane * 16, mr + m0);
@@ -617,7 +623,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         for (int tt = 0; tt < NTL; ++tt) {
           uint16_t* wbt = wb + (t_first + tt) * C::WB_HALVES;
 #pragma unroll
-          for (int gr = 0; gr < NG; ++gr) {
+          for (int gr = 0; gr < NGV; ++gr) {
             const float2 sc = scales_of(vpa[tt][gr], vpb[tt][gr]);
             const float2 zr = zeros_of(vpa[tt][gr], vpb[tt][gr]);
 #pragma unroll
@@ -649,17 +655,17 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         }
       }
       // ---- output: O^T[dim][col] += codes^T . (p * scale_v)
-      uint32_t bp[NTL][NP][NG][2];
+      uint32_t bp[NTL][NP][NGV][2];
       uint32_t vw[NTL][C::VW];
 #pragma unroll
       for (int tt = 0; tt < NTL; ++tt) {
         if constexpr (QS == 2) {
           // transposed loads give the B fragments (tokens 2c, 2c+1 | +8, +9; column g)
           const uint8_t* wbt = reinterpret_cast<const uint8_t*>(wb + (t_first + tt) * C::WB_HALVES);
-          uint32_t d[2 * NG * NP];
+          uint32_t d[2 * NGV * NP];
 #pragma unroll
-          for (int m0 = 0; m0 < 2 * NG * NP; m0 += 4) {
-            if constexpr (2 * NG * NP >= 4)
+          for (int m0 = 0; m0 < 2 * NGV * NP; m0 += 4) {
+            if constexpr (2 * NGV * NP >= 4)
               ldmatrix_trans_b16<4>(wbt + m0 * 128 + lane * 16, d + m0);
             else
               ldmatrix_trans_b16<2>(wbt + m0 * 128 + lane * 16, d + m0);
@@ -667,16 +673,16 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
 #pragma unroll
           for (int pt = 0; pt < NP; ++pt)
 #pragma unroll
-            for (int gr = 0; gr < NG; ++gr) {
-              bp[tt][pt][gr][0] = d[2 * (pt * NG + gr)];
-              bp[tt][pt][gr][1] = d[2 * (pt * NG + gr) + 1];
+            for (int gr = 0; gr < NGV; ++gr) {
+              bp[tt][pt][gr][0] = d[2 * (pt * NGV + gr)];
+              bp[tt][pt][gr][1] = d[2 * (pt * NGV + gr) + 1];
             }
         } else {
           const uint16_t* rd = wb + (t_first + tt) * C::WB_HALVES + g * C::WB_RS + 2 * c;
 #pragma unroll
           for (int pt = 0; pt < NP; ++pt)
 #pragma unroll
-            for (int gr = 0; gr < NG; ++gr) {
+            for (int gr = 0; gr < NGV; ++gr) {
               const uint16_t* row = rd + (gr * 8 + 4 * pt) * 2 * C::WB_RS;
               bp[tt][pt][gr][0] = *reinterpret_cast<const uint32_t*>(row);
               bp[tt][pt][gr][1] = *reinterpret_cast<const uint32_t*>(row + 8);
@@ -689,7 +695,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       }
 #pragma unroll
       for (int j = 0; j < KSTEPS; ++j) {
-        const int gr = 16 * j / G;
+        const int gr = 16 * j / GV;
 #pragma unroll
         for (int tt = 0; tt < NTL; ++tt) {
           const uint32_t a0 = extract_codes<C::BV>(vw[tt], 0, 2 * j);
@@ -750,8 +756,8 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   float* ob = reinterpret_cast<float*>(smem);  // [warp][8][D]
   float* mb = mrg;                             // [warp][8]
   float* lb = mb + C::kWarps * 8;              // [warp][8]
-  float* zb = lb + C::kWarps * 8;              // [warp][8][NG]
-  float* wt = zb + C::kWarps * 8 * NG;         // [head][warp] merge weights
+  float* zb = lb + C::kWarps * 8;              // [warp][8][NGV]
+  float* wt = zb + C::kWarps * 8 * NGV;         // [head][warp] merge weights
   float* rden = wt + 8 * C::kWarps;            // [head] 1 / denominator
   {
 #pragma unroll
@@ -761,9 +767,9 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       l += __shfl_xor_sync(0xffffffffu, l, 4);
       l += __shfl_xor_sync(0xffffffffu, l, 8);
       l += __shfl_xor_sync(0xffffffffu, l, 16);
-      float z[NG];
+      float z[NGV];
 #pragma unroll
-      for (int gr = 0; gr < NG; ++gr) {
+      for (int gr = 0; gr < NGV; ++gr) {
         z[gr] = zacc[hs][gr].x + zacc[hs][gr].y;
         z[gr] += __shfl_xor_sync(0xffffffffu, z[gr], 4);
         z[gr] += __shfl_xor_sync(0xffffffffu, z[gr], 8);
@@ -773,7 +779,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         mb[warp * 8 + head] = m_run[hs];
         lb[warp * 8 + head] = l;
 #pragma unroll
-        for (int gr = 0; gr < NG; ++gr) zb[(warp * 8 + head) * NG + gr] = z[gr];
+        for (int gr = 0; gr < NGV; ++gr) zb[(warp * 8 + head) * NGV + gr] = z[gr];
       }
     }
 #pragma unroll
@@ -814,7 +820,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     float num = 0.0f;
 #pragma unroll
     for (int w = 0; w < C::kWarps; ++w)
-      num = fmaf(wt[head * C::kWarps + w], ob[(w * 8 + head) * D + d] + zb[(w * 8 + head) * NG + d / G], num);
+      num = fmaf(wt[head * C::kWarps + w], ob[(w * 8 + head) * D + d] + zb[(w * 8 + head) * NGV + d / GV], num);
     if (direct) {
       store_out(a.out, a.out_dtype, (static_cast<size_t>(b) * a.q_heads + head0 + head) * D + d,
                 num * rden[head]);
@@ -840,28 +846,38 @@ DecodeKernel make_decode_kernel() {
   return k;
 }
 
-// Instances for one (bits_k, bits_v) pair: D in {64, 128}, groups per row,
-// and the query variants: up to 4 heads per CTA (any query type: one head per
-// lane, high/low columns), 5..8 heads with 16-bit queries (two heads per
-// lane), 5..8 heads with binary32 queries (high/low columns, two n-tiles).
+// Instances for one (bits_k, bits_v) pair: D in {64, 128}; groups per row of
+// keys and values, equal or with finer key groups (the page's group-size
+// finding: keys gain from smaller groups, values do not need them); and the
+// query variants: up to 4 heads per CTA (any query type: one head per lane,
+// high/low columns), 5..8 heads with 16-bit queries (two heads per lane),
+// 5..8 heads with binary32 queries (high/low columns, two n-tiles).
 template <int BK, int BV>
-bool get_decode_kernel_bits(int head_dim, int num_groups, int variant, DecodeKernel* out) {
-#define KVQ_VARIANTS(D, NG)                                                        \
-  switch (variant) {                                                               \
-    case 0:                                                                        \
-    case 1: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NG, 2, 1, 1>>(); return true; \
-    case 2: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NG, 1, 1, 2>>(); return true; \
-    case 3: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NG, 2, 2, 2>>(); return true; \
-    default: return false;                                                         \
+bool get_decode_kernel_bits(int head_dim, int groups_k, int groups_v, int variant,
+                            DecodeKernel* out) {
+#define KVQ_VARIANTS(D, NGK, NGV)                                                          \
+  switch (variant) {                                                                       \
+    case 0:                                                                                \
+    case 1: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NGK, NGV, 2, 1, 1>>(); return true; \
+    case 2: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NGK, NGV, 1, 1, 2>>(); return true; \
+    case 3: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NGK, NGV, 2, 2, 2>>(); return true; \
+    default: return false;                                                                 \
   }
+#define KVQ_GROUPS(D, NGK, NGV) \
+  if (groups_k == NGK && groups_v == NGV) { KVQ_VARIANTS(D, NGK, NGV) }
   if (head_dim == 128) {
-    if (num_groups == 1) { KVQ_VARIANTS(128, 1) }
-    if (num_groups == 2) { KVQ_VARIANTS(128, 2) }
-    if (num_groups == 4) { KVQ_VARIANTS(128, 4) }
+    KVQ_GROUPS(128, 1, 1)
+    KVQ_GROUPS(128, 2, 2)
+    KVQ_GROUPS(128, 4, 4)
+    KVQ_GROUPS(128, 2, 1)
+    KVQ_GROUPS(128, 4, 2)
+    KVQ_GROUPS(128, 4, 1)
   } else if (head_dim == 64) {
-    if (num_groups == 1) { KVQ_VARIANTS(64, 1) }
-    if (num_groups == 2) { KVQ_VARIANTS(64, 2) }
+    KVQ_GROUPS(64, 1, 1)
+    KVQ_GROUPS(64, 2, 2)
+    KVQ_GROUPS(64, 2, 1)
   }
+#undef KVQ_GROUPS
 #undef KVQ_VARIANTS
   return false;
 }

@@ -2,7 +2,8 @@
 #include "decode.cuh"
 
 namespace kvq {
-bool get_decode_kernel_k8v8(int head_dim, int num_groups, int variant, DecodeKernel* out) {
-  return get_decode_kernel_bits<8, 8>(head_dim, num_groups, variant, out);
+bool get_decode_kernel_k8v8(int head_dim, int groups_k, int groups_v, int variant,
+                            DecodeKernel* out) {
+  return get_decode_kernel_bits<8, 8>(head_dim, groups_k, groups_v, variant, out);
 }
 }  // namespace kvq

@@ -39,6 +39,7 @@ struct QuantizeArgs {
   const int32_t* pos;
   int n_new;
   int batch, kv_heads, head_dim, capacity, bits_k, bits_v, group;
+  int group_v;       // values' group size
   uint32_t* err;
   bool rotate_keys;  // store keys as H k (Walsh-Hadamard along head_dim)
 };
@@ -81,9 +82,9 @@ struct DecodeKernel {
   cudaError_t (*launch)(const DecodeArgs&, dim3 grid, cudaStream_t stream);
 };
 
-// Returns false if (D, bits_k, bits_v, groups, variant) has no instance.
-bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int num_groups, int variant,
-                       DecodeKernel* out);
+// Returns false if (D, bits, key groups, value groups, variant) has no instance.
+bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int groups_k, int groups_v,
+                       int variant, DecodeKernel* out);
 
 struct CombineArgs {
   const float* ws_o;

@@ -35,10 +35,11 @@
 
 namespace kvq {
 
-template <int D_, int BK_, int BV_, int G_>
+// GK / GV: group sizes of the keys / values.
+template <int D_, int BK_, int BV_, int GK_, int GV_>
 struct QCfg {
-  static constexpr int D = D_, BK = BK_, BV = BV_, G = G_;
-  static constexpr int NG = D / G;
+  static constexpr int D = D_, BK = BK_, BV = BV_, GK = GK_, GV = GV_;
+  static constexpr int NGK = D / GK, NGV = D / GV;
   static constexpr int EK = 16 / BK, EV = 16 / BV;
   static constexpr int CHK = 8 * EK, CHV = 8 * EV;  // elements per chunk
   static constexpr int CK = D / CHK, CV = D / CHV;  // chunks per token
@@ -51,7 +52,7 @@ struct QCfg {
   static constexpr int VN = D * BV / 16;
   static constexpr int VP = VN < 16 ? VN : 16;
   static constexpr int WV = D * BV / 128;
-  static_assert(G % 8 == 0 && D % CHK == 0 && D % CHV == 0, "shape");
+  static_assert(GK % 8 == 0 && GV % 8 == 0 && D % CHK == 0 && D % CHV == 0, "shape");
 };
 
 // Raw input pairs and their conversions.
@@ -240,12 +241,12 @@ __device__ __forceinline__ void rotate_row_chunk(float2 (&f)[CH / 2], int w) {
 
 template <class C, typename TIn, bool ROT>
 __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const QuantizeArgs a) {
-  constexpr int D = C::D, G = C::G, NG = C::NG;
+  constexpr int D = C::D, NGK = C::NGK, NGV = C::NGV;
   using P = InPair<TIn>;
   __shared__ __align__(16) uint8_t sk[16 * C::KROW];
   __shared__ __align__(16) uint8_t sv[C::VTILE];
-  __shared__ __align__(16) uint32_t skp[16 * NG];
-  __shared__ __align__(16) uint32_t svp[16 * NG];
+  __shared__ __align__(16) uint32_t skp[16 * NGK];
+  __shared__ __align__(16) uint32_t svp[16 * NGV];
 
   const int b = blockIdx.z;
   const int h = blockIdx.y;
@@ -286,20 +287,20 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
       for (int i = 0; i < CH / 2; ++i) raw[i] = P::zero();
     }
     uint32_t acc[8];
-    uint32_t par[CH / G > 0 ? CH / G : 1];
+    uint32_t par[CH / C::GK > 0 ? CH / C::GK : 1];
     if constexpr (ROT) {
       // rotated keys: quantize H k, computed in binary32 (exact widening first)
       float2 f[CH / 2];
 #pragma unroll
       for (int i = 0; i < CH / 2; ++i) f[i] = P::to_f2(raw[i]);
       rotate_row_chunk<CH, C::CK>(f, w);
-      quantize_chunk<C::BK, G, CH, float>(f, acc, par);
+      quantize_chunk<C::BK, C::GK, CH, float>(f, acc, par);
     } else {
-      quantize_chunk<C::BK, G, CH, TIn>(raw, acc, par);
+      quantize_chunk<C::BK, C::GK, CH, TIn>(raw, acc, par);
     }
-    constexpr int NPAR = CH / G > 0 ? CH / G : 1;
-    const bool reports = G > CH ? (w % (G / CH)) == 0 : true;
-    const int first_group = (CH * w) / G;
+    constexpr int NPAR = CH / C::GK > 0 ? CH / C::GK : 1;
+    const bool reports = C::GK > CH ? (w % (C::GK / CH)) == 0 : true;
+    const int first_group = (CH * w) / C::GK;
     if (full_tile && k < 16) {
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
             __byte_perm(acc[2 * c], acc[2 * c + 1], 0x5410);
       if (reports)
 #pragma unroll
-        for (int q = 0; q < NPAR; ++q) skp[k * NG + first_group + q] = par[q];
+        for (int q = 0; q < NPAR; ++q) skp[k * NGK + first_group + q] = par[q];
     } else if (valid) {
       uint8_t* row = a.k_codes + (slot * a.capacity + p) * C::KROW;
 #pragma unroll
@@ -317,7 +318,7 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
       if (reports)
 #pragma unroll
         for (int q = 0; q < NPAR; ++q)
-          a.k_params[(slot * a.capacity + p) * NG + first_group + q] = par[q];
+          a.k_params[(slot * a.capacity + p) * NGK + first_group + q] = par[q];
     }
   } else {
     // ---------------------------------------------------------- values
@@ -333,11 +334,11 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
       for (int i = 0; i < CH / 2; ++i) raw[i] = P::zero();
     }
     uint32_t acc[8];
-    uint32_t par[CH / G > 0 ? CH / G : 1];
-    quantize_chunk<C::BV, G, CH, TIn>(raw, acc, par);
-    constexpr int NPAR = CH / G > 0 ? CH / G : 1;
-    const bool reports = G > CH ? (w % (G / CH)) == 0 : true;
-    const int first_group = (CH * w) / G;
+    uint32_t par[CH / C::GV > 0 ? CH / C::GV : 1];
+    quantize_chunk<C::BV, C::GV, CH, TIn>(raw, acc, par);
+    constexpr int NPAR = CH / C::GV > 0 ? CH / C::GV : 1;
+    const bool reports = C::GV > CH ? (w % (C::GV / CH)) == 0 : true;
+    const int first_group = (CH * w) / C::GV;
     // half-word of position k in lane 4g + (k mod 8)/2, word (k/8)*WV + w
     const int n = 4 * ((k / 8) * C::WV + w) + 2 * (k % 2);
     const int lane0 = (k % 8) / 2;
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
         *reinterpret_cast<uint16_t*>(sv + off0 + 4 * g * C::VP) = static_cast<uint16_t>(acc[g]);
       if (reports)
 #pragma unroll
-        for (int q = 0; q < NPAR; ++q) svp[k * NG + first_group + q] = par[q];
+        for (int q = 0; q < NPAR; ++q) svp[k * NGV + first_group + q] = par[q];
     } else if (valid) {
       uint8_t* gt = a.v_codes + (slot * (a.capacity / 16) + tile) * C::VTILE;
 #pragma unroll
@@ -357,7 +358,7 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
       if (reports)
 #pragma unroll
         for (int q = 0; q < NPAR; ++q)
-          a.v_params[(slot * a.capacity + p) * NG + first_group + q] = par[q];
+          a.v_params[(slot * a.capacity + p) * NGV + first_group + q] = par[q];
     }
   }
 
@@ -365,50 +366,58 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
     __syncthreads();
     uint4* gk = reinterpret_cast<uint4*>(a.k_codes + (slot * a.capacity + tile * 16) * C::KROW);
     uint4* gv = reinterpret_cast<uint4*>(a.v_codes + (slot * (a.capacity / 16) + tile) * C::VTILE);
-    uint4* gkp = reinterpret_cast<uint4*>(a.k_params + (slot * a.capacity + tile * 16) * NG);
-    uint4* gvp = reinterpret_cast<uint4*>(a.v_params + (slot * a.capacity + tile * 16) * NG);
+    uint4* gkp = reinterpret_cast<uint4*>(a.k_params + (slot * a.capacity + tile * 16) * NGK);
+    uint4* gvp = reinterpret_cast<uint4*>(a.v_params + (slot * a.capacity + tile * 16) * NGV);
     for (int i = t; i < 16 * C::KROW / 16; i += C::THREADS) gk[i] = reinterpret_cast<const uint4*>(sk)[i];
     for (int i = t; i < C::VTILE / 16; i += C::THREADS) gv[i] = reinterpret_cast<const uint4*>(sv)[i];
-    for (int i = t; i < NG * 4; i += C::THREADS) {  // 16 * NG words = 4 * NG uint4
+    for (int i = t; i < NGK * 4; i += C::THREADS)  // 16 * NGK words = 4 * NGK uint4
       gkp[i] = reinterpret_cast<const uint4*>(skp)[i];
+    for (int i = t; i < NGV * 4; i += C::THREADS)
       gvp[i] = reinterpret_cast<const uint4*>(svp)[i];
-    }
   }
 }
 
-template <int D, int BK, int BV, int G, typename TIn>
+template <int D, int BK, int BV, int GK, int GV, typename TIn>
 cudaError_t launch_q(const QuantizeArgs& a, cudaStream_t stream) {
-  using C = QCfg<D, BK, BV, G>;
+  using C = QCfg<D, BK, BV, GK, GV>;
   const dim3 grid((a.n_new + 30) / 16, a.kv_heads, a.batch);
   if (a.rotate_keys)
     return launch_pdl(quantize_append_kernel<C, TIn, true>, grid, dim3(C::THREADS), 0, stream, a);
   return launch_pdl(quantize_append_kernel<C, TIn, false>, grid, dim3(C::THREADS), 0, stream, a);
 }
 
-// Dispatch over (D, G, bits) for one input type.
+// Dispatch over (D, key and value groups, bits) for one input type: equal
+// groups, or coarser value groups (the combinations the decode kernel has).
 template <typename TIn>
 cudaError_t launch_quantize_typed(const QuantizeArgs& a, cudaStream_t stream) {
-#define KVQ_Q_BITS(D, G)                                                            \
+#define KVQ_Q_BITS(D, GK, GV)                                                       \
   switch (a.bits_k * 16 + a.bits_v) {                                                \
-    case 0x22: return launch_q<D, 2, 2, G, TIn>(a, stream);                          \
-    case 0x24: return launch_q<D, 2, 4, G, TIn>(a, stream);                          \
-    case 0x28: return launch_q<D, 2, 8, G, TIn>(a, stream);                          \
-    case 0x42: return launch_q<D, 4, 2, G, TIn>(a, stream);                          \
-    case 0x44: return launch_q<D, 4, 4, G, TIn>(a, stream);                          \
-    case 0x48: return launch_q<D, 4, 8, G, TIn>(a, stream);                          \
-    case 0x82: return launch_q<D, 8, 2, G, TIn>(a, stream);                          \
-    case 0x84: return launch_q<D, 8, 4, G, TIn>(a, stream);                          \
-    case 0x88: return launch_q<D, 8, 8, G, TIn>(a, stream);                          \
+    case 0x22: return launch_q<D, 2, 2, GK, GV, TIn>(a, stream);                     \
+    case 0x24: return launch_q<D, 2, 4, GK, GV, TIn>(a, stream);                     \
+    case 0x28: return launch_q<D, 2, 8, GK, GV, TIn>(a, stream);                     \
+    case 0x42: return launch_q<D, 4, 2, GK, GV, TIn>(a, stream);                     \
+    case 0x44: return launch_q<D, 4, 4, GK, GV, TIn>(a, stream);                     \
+    case 0x48: return launch_q<D, 4, 8, GK, GV, TIn>(a, stream);                     \
+    case 0x82: return launch_q<D, 8, 2, GK, GV, TIn>(a, stream);                     \
+    case 0x84: return launch_q<D, 8, 4, GK, GV, TIn>(a, stream);                     \
+    case 0x88: return launch_q<D, 8, 8, GK, GV, TIn>(a, stream);                     \
     default: return cudaErrorInvalidValue;                                           \
   }
+#define KVQ_Q_GROUPS(D, GK, GV) \
+  if (a.group == GK && a.group_v == GV) { KVQ_Q_BITS(D, GK, GV) }
   if (a.head_dim == 128) {
-    if (a.group == 32) { KVQ_Q_BITS(128, 32) }
-    if (a.group == 64) { KVQ_Q_BITS(128, 64) }
-    if (a.group == 128) { KVQ_Q_BITS(128, 128) }
+    KVQ_Q_GROUPS(128, 32, 32)
+    KVQ_Q_GROUPS(128, 64, 64)
+    KVQ_Q_GROUPS(128, 128, 128)
+    KVQ_Q_GROUPS(128, 32, 64)
+    KVQ_Q_GROUPS(128, 32, 128)
+    KVQ_Q_GROUPS(128, 64, 128)
   } else {
-    if (a.group == 32) { KVQ_Q_BITS(64, 32) }
-    if (a.group == 64) { KVQ_Q_BITS(64, 64) }
+    KVQ_Q_GROUPS(64, 32, 32)
+    KVQ_Q_GROUPS(64, 64, 64)
+    KVQ_Q_GROUPS(64, 32, 64)
   }
+#undef KVQ_Q_GROUPS
 #undef KVQ_Q_BITS
   return cudaErrorInvalidValue;
 }

@@ -55,7 +55,7 @@ def test_cache_bytes_rejects_bad_shapes(args):
 
 def _desc(**kw):
     d = dict(batch=1, kv_heads=2, head_dim=128, capacity=64, bits_k=4, bits_v=2, group=64,
-             flags=0, k_codes=0x1000, v_codes=0x2000, k_params=0x3000, v_params=0x4000)
+             flags=0, group_v=0, reserved=0, k_codes=0x1000, v_codes=0x2000, k_params=0x3000, v_params=0x4000)
     d.update(kw)
     return kvq.KvqCacheDesc(*d.values())
 
@@ -67,6 +67,12 @@ def test_validate_cache_host_only():
     assert lib.kvq_validate_cache(ctypes.byref(_desc(v_params=0))) == kvq.KVQ_ERR_INVALID_ARG
     assert lib.kvq_validate_cache(ctypes.byref(_desc(flags=kvq.KVQ_FLAG_ROTATE_KEYS))) == kvq.KVQ_OK
     assert lib.kvq_validate_cache(ctypes.byref(_desc(flags=2))) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_validate_cache(ctypes.byref(_desc(reserved=1))) == kvq.KVQ_ERR_INVALID_ARG
+    # value groups: equal or coarser than the keys' (group 64 here)
+    assert lib.kvq_validate_cache(ctypes.byref(_desc(group_v=128))) == kvq.KVQ_OK
+    assert lib.kvq_validate_cache(ctypes.byref(_desc(group_v=64))) == kvq.KVQ_OK
+    assert lib.kvq_validate_cache(ctypes.byref(_desc(group_v=32))) == kvq.KVQ_ERR_UNSUPPORTED
+    assert lib.kvq_validate_cache(ctypes.byref(_desc(group_v=48))) == kvq.KVQ_ERR_UNSUPPORTED
     assert lib.kvq_validate_cache(ctypes.byref(_desc(bits_v=3))) == kvq.KVQ_ERR_UNSUPPORTED
     assert lib.kvq_validate_cache(ctypes.byref(_desc(capacity=24))) == kvq.KVQ_ERR_INVALID_ARG
     assert lib.kvq_validate_cache(None) == kvq.KVQ_ERR_INVALID_ARG
