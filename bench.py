@@ -15,6 +15,7 @@ by a barrier and a device synchronize, timed with CUDA events on the launch
 stream, max over ranks.  Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--bits K,V] [--group-v G] [--rotate-keys]
 """
 from __future__ import annotations
 

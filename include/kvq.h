@@ -12,7 +12,8 @@
  * plainest reading that the rest of the page supports:
  *
  *   * group-wise, uniform, asymmetric min-max quantization along head_dim,
- *     one (scale, zero) pair per group of `group` consecutive elements, stored
+ *     one (scale, zero) pair per group of `group` (keys) or `group_v`
+ *     (values) consecutive elements, stored
  *     as IEEE binary16 (the page's "group size" knob, section "Results",
  *     "Group-size sensitivity");
  *   * b-bit codes, b in {2, 4, 8}, bit-packed (the page's K4V2 / K2V4 /

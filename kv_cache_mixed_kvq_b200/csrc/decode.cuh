@@ -10,9 +10,12 @@
 // Design (B200, sm_100a):
 //  * each of the CTA's four warps runs its own copy pipeline: lane 0 streams
 //    the warp's next 32 positions of the four cache arrays into a ring of
-//    2-3 shared-memory slots with 1-D bulk copies (cp.async.bulk, no
+//    two shared-memory slots with 1-D bulk copies (cp.async.bulk, no
 //    multicast) counted on the warp's own mbarriers (bounded waits), and the
 //    warp processes its two 16-token tiles phase by phase;
+//  * keys and values may have different group sizes (NGK, NGV groups per
+//    row): the score side uses the key groups, the output side the value
+//    groups;
 //  * codes stay integers: every code becomes an exact binary16 subnormal
 //    (code * 2^(pos-24)) with one AND, so tensor cores (mma.sync m16n8k16,
 //    fp32 accumulate) multiply raw codes; the per-group scale and zero are
@@ -24,7 +27,10 @@
 //    output product) are split the same way and scaled per warp by a power of
 //    two, so products keep ~22 bits;
 //  * online softmax in binary32 (exp2 domain) with a lazily updated maximum;
-//    partial results per split are merged by a separate log-sum-exp combine.
+//    partial results per split are merged by a separate log-sum-exp combine,
+//    except when a row has a single split: its CTA then writes the output;
+//  * with rotated keys (KVQ_FLAG_ROTATE_KEYS) the prologue turns the query
+//    into H q / D in shared memory.
 #pragma once
 
 #include <type_traits>

@@ -2,7 +2,8 @@
 // new K/V rows into the packed cache ("Quantize What Counts: More for Keys,
 // Less for Values", summary page, "Problem statement" / "Key contributions":
 // keys at b_k bits, values at b_v bits; "Results", "Group-size sensitivity":
-// one scale/zero per group of head_dim elements).
+// one scale/zero per group of head_dim elements; keys and values may use
+// different group sizes, GK and GV).
 //
 // One CTA handles one 16-position tile of one (batch row, kv head) slot;
 // each thread issues all its 16-byte loads before any arithmetic, and about
