@@ -70,10 +70,15 @@ def algorithmic_bytes(w: workloads.Workload, bits, n_new, read_lens, group_v: in
 
 
 def sha_of(paths):
+    """Hash of the code in `paths` (line comments and blank lines removed, so
+    that comment-only edits keep recorded counters valid)."""
     h = hashlib.sha256()
     for p in paths:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p)) as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 
