@@ -143,3 +143,22 @@ def as_bits(t: torch.Tensor):
     if t.dtype == torch.float16:
         return t.view(torch.int16).numpy().view("uint16"), "f16"
     raise TypeError(t.dtype)
+
+
+def make_block_table(lens, capacity: int, page_size: int, seed: int = 0, spare: int = 0):
+    """Seeded block table for a paged cache: each row gets ceil(len / P) pages,
+    drawn without repetition from a shuffled pool of exactly that many pages
+    plus `spare` unused ones (fragmented placement, as after many
+    allocations and frees); entries past a row's length are -1.  Returns
+    (int32 numpy [len(lens)][capacity / P], num_pages)."""
+    import numpy as np
+
+    need = [(int(n) + page_size - 1) // page_size for n in lens]
+    num_pages = max(1, sum(need) + spare)
+    order = np.random.default_rng(seed).permutation(num_pages)
+    table = np.full((len(lens), capacity // page_size), -1, np.int32)
+    i = 0
+    for b, n in enumerate(need):
+        table[b, :n] = order[i:i + n]
+        i += n
+    return table, num_pages

@@ -213,6 +213,118 @@ class HostCache:
         return out, r
 
 
+DEVERR_CAPACITY, DEVERR_BAD_POS, DEVERR_BAD_PAGE = 1, 8, 16
+
+
+class PagedHostCache:
+    """Paged variant (block tables) of HostCache.
+
+    The summary page has no paged layout: this is the serving-system variant
+    of the cache format, defined by its mapping alone.  A pool of
+    ``num_pages`` pages of ``page_size`` (P) positions holds all kv heads of
+    each page, and (page, kv head) is laid out exactly like a slot of P
+    positions, so the pool is a HostCache of ``num_pages`` batch rows and
+    capacity P.  Position p of batch row b is local position p mod P of page
+    ``block_table[b][p // P]``.
+
+    Every operation gathers each batch row's pages into a slot-layout
+    HostCache of ``capacity`` positions, runs the slot operation there and
+    scatters the pages back (batch rows one after another).  Block-table
+    entries outside [0, num_pages) read as zero pages and are never written;
+    reaching one sets DEVERR_BAD_PAGE.
+    """
+
+    def __init__(self, B, Hkv, D, capacity, bits_k, bits_v, group, page_size, num_pages,
+                 block_table, rotate_keys=False, group_v=None):
+        assert capacity % page_size == 0 and page_size % 16 == 0
+        self.B, self.Hkv, self.D, self.cap, self.P = B, Hkv, D, capacity, page_size
+        self.num_pages = num_pages
+        self.shape = (D, bits_k, bits_v, group, rotate_keys, group_v)
+        self.block_table = np.array(block_table, dtype=np.int64).reshape(B, capacity // page_size)
+        self.pool = HostCache(num_pages, Hkv, D, page_size, bits_k, bits_v, group,
+                              rotate_keys=rotate_keys, group_v=group_v)
+
+    # the four arrays, page-major [num_pages][Hkv][...]
+    @property
+    def arrays(self):
+        p = self.pool
+        return [p.k_codes, p.v_codes, p.k_params, p.v_params]
+
+    def _row_cache(self, rows: int) -> HostCache:
+        D, bk, bv, g, rot, gv = self.shape
+        return HostCache(rows, self.Hkv, D, self.cap, bk, bv, g, rotate_keys=rot, group_v=gv)
+
+    def _views(self, hc: HostCache, rows: int):
+        """(pool view [num_pages][Hkv][L], row view [rows][Hkv][pages per row][L])
+        of each array, L the elements of P positions of one slot."""
+        npg = self.cap // self.P
+        out = []
+        for pool_a, row_a in zip(self.arrays, (hc.k_codes, hc.v_codes, hc.k_params, hc.v_params)):
+            L = pool_a.size // (self.num_pages * self.Hkv)
+            out.append((pool_a.reshape(self.num_pages, self.Hkv, L),
+                        row_a.reshape(rows, self.Hkv, npg, L)))
+        return out
+
+    def _valid(self, page) -> bool:
+        return 0 <= page < self.num_pages
+
+    def gather(self, rows=None) -> HostCache:
+        """Slot-layout copy of the given batch rows (all by default)."""
+        rows = list(range(self.B)) if rows is None else list(rows)
+        hc = self._row_cache(len(rows))
+        for pool_v, row_v in self._views(hc, len(rows)):
+            for i, b in enumerate(rows):
+                for j, page in enumerate(self.block_table[b]):
+                    if self._valid(page):
+                        row_v[i, :, j, :] = pool_v[page]
+        return hc
+
+    def _scatter(self, hc: HostCache, b: int, pages) -> None:
+        for pool_v, row_v in self._views(hc, 1):
+            for j in pages:
+                page = self.block_table[b][j]
+                if self._valid(page):
+                    pool_v[page] = row_v[0, :, j, :]
+
+    def quantize_append(self, k: np.ndarray, v: np.ndarray, pos, dtype: str | None = None) -> int:
+        """As HostCache.quantize_append, through the block table."""
+        k = np.ascontiguousarray(k)
+        v = np.ascontiguousarray(v)
+        n_new = k.shape[2]
+        flags = 0
+        for b in range(self.B):
+            hc = self.gather([b])
+            r = hc.quantize_append(k[b:b + 1], v[b:b + 1], [int(pos[b])], dtype=dtype)
+            flags |= r
+            if r & (DEVERR_CAPACITY | DEVERR_BAD_POS) or n_new == 0:
+                continue  # row rejected: nothing written, no page reached
+            first = (int(pos[b]) // 16) * 16
+            last = (int(pos[b]) + n_new + 15) // 16 * 16 - 1  # last position of the last tile
+            pages = range(first // self.P, last // self.P + 1)
+            if any(not self._valid(self.block_table[b][j]) for j in pages):
+                flags |= DEVERR_BAD_PAGE
+            self._scatter(hc, b, pages)
+        return flags
+
+    def decode_attention(self, q: np.ndarray, Hq: int, seq_lens, sm_scale: float = 0.0,
+                         q_dtype: str | None = None, max_len: int | None = None):
+        """As HostCache.decode_attention over the gathered rows; rows that
+        reach an invalid page set DEVERR_BAD_PAGE (their output is not
+        defined by the library)."""
+        out, flags = self.gather().decode_attention(q, Hq, seq_lens, sm_scale=sm_scale,
+                                                    q_dtype=q_dtype, max_len=max_len)
+        lim = min(self.cap, self.cap if max_len is None else max_len)
+        for b, n in enumerate(seq_lens):
+            n = max(0, min(int(n), lim))
+            if any(not self._valid(self.block_table[b][j]) for j in range((n + self.P - 1) // self.P)):
+                flags |= DEVERR_BAD_PAGE
+        return out, flags
+
+    def dequant_row(self, which: int, b: int, h: int, p: int) -> np.ndarray:
+        page = int(self.block_table[b][p // self.P])
+        return self.pool.dequant_row(which, page, h, p % self.P)
+
+
 def fwht(x) -> np.ndarray:
     """Unnormalised Walsh-Hadamard transform of a binary32 vector (the oracle's
     key rotation, same butterfly order and rounding)."""
