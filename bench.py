@@ -182,7 +182,7 @@ class Arm:
     """Device buffers for R rotating sets of inputs + caches, and the step."""
 
     def __init__(self, w, bits, rotate: int, device, rotate_keys: bool = False,
-                 group_v: int = 0):
+                 group_v: int = 0, page_size: int = 0):
         import kv_cache_mixed_kvq_b200 as kvq
         self.kvq = kvq
         self.w, self.bits = w, bits
@@ -192,10 +192,19 @@ class Arm:
         self.max_len = max(self.read)
         self.pos_t = torch.tensor(self.pos, dtype=torch.int32, device=device)
         self.sets = []
+        self.page_size = page_size
         for r in range(rotate):
+            paged = {}
+            if page_size:
+                # a pool of exactly the pages the rows use, shuffled (fragmented)
+                need = [max(self.read[b], self.pos[b] + self.n_new) for b in range(w.batch)]
+                table, num_pages = workloads.make_block_table(need, self.cap, page_size,
+                                                              seed=7 + r)
+                paged = dict(page_size=page_size, num_pages=num_pages,
+                             block_table=torch.from_numpy(table))
             cache = kvq.KVCache.allocate(w.batch, w.kv_heads, w.head_dim, self.cap, bits[0],
                                          bits[1], w.group, device=device,
-                                         rotate_keys=rotate_keys, group_v=group_v)
+                                         rotate_keys=rotate_keys, group_v=group_v, **paged)
             if w.name != "llama3_8b":
                 # pre-fill the context (untimed); the step then appends n_new tokens
                 for b in range(w.batch):
@@ -234,6 +243,13 @@ class Arm:
 
 def _slot_view(cache, b):
     """A KVCache over batch row b only (views into the same buffers)."""
+    if cache.page_size:  # the whole pool, row b's block table
+        return type(cache)(1, cache.kv_heads, cache.head_dim, cache.capacity, cache.bits_k,
+                           cache.bits_v, cache.group, cache.k_codes, cache.v_codes,
+                           cache.k_params, cache.v_params, rotate_keys=cache.rotate_keys,
+                           group_v=cache.group_v, page_size=cache.page_size,
+                           num_pages=cache.num_pages,
+                           block_table=cache.block_table[b:b + 1].contiguous())
     per = [t.numel() // cache.batch for t in (cache.k_codes, cache.v_codes, cache.k_params,
                                                 cache.v_params)]
     return type(cache)(1, cache.kv_heads, cache.head_dim, cache.capacity, cache.bits_k,
@@ -248,7 +264,8 @@ def run_ours(args, rank, world, device):
     bits = tuple(int(x) for x in args.bits.split(",")) if args.bits else w.bits[-1] \
         if w.name == "long" else w.bits[0]
     rotate = args.rotate
-    arm = Arm(w, bits, rotate, device, rotate_keys=args.rotate_keys, group_v=args.group_v)
+    arm = Arm(w, bits, rotate, device, rotate_keys=args.rotate_keys, group_v=args.group_v,
+              page_size=args.page_size)
     stream = torch.cuda.current_stream()
 
     # warm-up (also loads every kernel and the error-word address)
@@ -334,6 +351,7 @@ def run_ours(args, rank, world, device):
             "bits_k": bits[0], "bits_v": bits[1], "group": w.group,
             "rotate_keys": bool(args.rotate_keys),
             "group_v": args.group_v or w.group,
+            "page_size": args.page_size,
             "step": ("quantize full cache + decode + combine" if w.name == "llama3_8b" else
                      f"append {arm.n_new} + decode + combine"),
             "split_tokens": arm.split_tokens,
@@ -536,6 +554,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--group-v", type=int, default=0,
                     help="values' group size (default: the workload's group)")
+    ap.add_argument("--page-size", type=int, default=0,
+                    help="paged cache layout with pages of this many positions (0: slots)")
     ap.add_argument("--rotate-keys", action="store_true",
                     help="cache with key-only Walsh-Hadamard rotation (KVQ_FLAG_ROTATE_KEYS)")
     args = ap.parse_args()

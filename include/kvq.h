@@ -126,7 +126,8 @@ enum kvq_device_error {
   KVQ_DEVERR_CAPACITY = 1u,    /* append with pos + n_new > capacity (rows skipped)   */
   KVQ_DEVERR_SEQ_LEN = 2u,     /* seq_lens[b] > max_seq_len or capacity (clamped)     */
   KVQ_DEVERR_TIMEOUT = 4u,     /* a bounded shared-memory pipeline wait gave up       */
-  KVQ_DEVERR_BAD_POS = 8u      /* pos[b] < 0 (rows skipped)                            */
+  KVQ_DEVERR_BAD_POS = 8u,     /* pos[b] < 0 (rows skipped)                            */
+  KVQ_DEVERR_BAD_PAGE = 16u    /* block_table entry outside [0, num_pages) (see below) */
 };
 
 /* Bits of kvq_cache_desc.flags. */
@@ -141,7 +142,15 @@ enum kvq_cache_flags {
    * the groups, scales and zeros then apply to H k.  Decode multiplies the
    * query by H / D, so scores are unchanged in exact arithmetic
    * ((H q / D) . (H k) = q . k).  Values are never rotated. */
-  KVQ_FLAG_ROTATE_KEYS = 1
+  KVQ_FLAG_ROTATE_KEYS = 1,
+  /* Paged layout (block tables): the cache is a pool of `num_pages` pages of
+   * `page_size` positions, and each batch row maps its logical positions to
+   * pages through `block_table`, so that ragged batches need no per-row
+   * capacity padding and rows can share pages (prefixes).  This is a
+   * serving-system variant of the cache format, not something the summary
+   * page describes; the codes, parameters and their placement inside a page
+   * are exactly those of the slot format above.  See kvq_cache_desc. */
+  KVQ_FLAG_PAGED = 2
 };
 
 /* Which array kvq_cache_bytes() sizes. */
@@ -163,6 +172,25 @@ enum kvq_cache_array {
  *   group <= group_v <= D ("Results", "Group-size sensitivity": finer
  *   groups help the keys, coarser ones are enough for the values).
  * Pointers: device memory, 16-byte aligned, sized by kvq_cache_bytes().
+ *
+ * Paged layout (flags & KVQ_FLAG_PAGED):
+ *   page_size (P): positions per page, a power of two >= 32 that divides
+ *     capacity; capacity is the logical length limit of every batch row.
+ *   num_pages: pages in the pool, >= 1.  A page holds P positions of all
+ *     kv_heads: the four arrays are page-major, [num_pages][Hkv][...], and
+ *     (page, h) is laid out exactly like a slot of capacity P above.  Size
+ *     them with kvq_cache_bytes(num_pages, kv_heads, head_dim, page_size,
+ *     ...).
+ *   block_table: device int32 [batch][capacity / P], 4-byte aligned:
+ *     positions [j*P, (j+1)*P) of batch row b live at local positions
+ *     0 .. P-1 of page block_table[b * (capacity / P) + j].  Entries that a
+ *     call never reaches are not read.  Rows may share pages for reading;
+ *     the pages one kvq_quantize_append() call writes must not be shared
+ *     between its batch rows (their writes would race).  An entry outside
+ *     [0, num_pages) that a call reaches flags KVQ_DEVERR_BAD_PAGE: an
+ *     append skips the 16-position tiles that map to it; decode attention
+ *     reads nothing from it and that row's output is unspecified.
+ * Without the flag, page_size and num_pages must be 0 and block_table NULL.
  */
 typedef struct kvq_cache_desc {
   int32_t batch;
@@ -179,12 +207,16 @@ typedef struct kvq_cache_desc {
   uint8_t* v_codes;
   void* k_params; /* binary16 (scale, zero) pairs */
   void* v_params; /* binary16 (scale, zero) pairs */
+  int32_t page_size;            /* KVQ_FLAG_PAGED: positions per page; else 0 */
+  int32_t num_pages;            /* KVQ_FLAG_PAGED: pages in the pool; else 0 */
+  const int32_t* block_table;   /* KVQ_FLAG_PAGED: [batch][capacity / page_size] */
 } kvq_cache_desc;
 
 /*
  * Bytes of one cache array for the given shape (all slots), or 0 if the
  * shape is invalid.  `group` is the group size of the array asked for: the
- * keys' for KVQ_K_PARAMS, the values' for KVQ_V_PARAMS.  Pure host function.
+ * keys' for KVQ_K_PARAMS, the values' for KVQ_V_PARAMS.  For a paged cache
+ * pass batch = num_pages and capacity = page_size.  Pure host function.
  */
 size_t kvq_cache_bytes(int32_t batch, int32_t kv_heads, int32_t head_dim,
                        int32_t capacity, int32_t bits_k, int32_t bits_v,

@@ -28,8 +28,9 @@ LIBRARY_PATH = os.path.join(_HERE, "libkvq.so")
 KVQ_F32, KVQ_BF16, KVQ_F16 = 0, 1, 2
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = range(5)
 KVQ_DEVERR_CAPACITY, KVQ_DEVERR_SEQ_LEN, KVQ_DEVERR_TIMEOUT, KVQ_DEVERR_BAD_POS = 1, 2, 4, 8
+KVQ_DEVERR_BAD_PAGE = 16
 KVQ_K_CODES, KVQ_V_CODES, KVQ_K_PARAMS, KVQ_V_PARAMS = range(4)
-KVQ_FLAG_ROTATE_KEYS = 1
+KVQ_FLAG_ROTATE_KEYS, KVQ_FLAG_PAGED = 1, 2
 
 _DTYPE = {torch.float32: KVQ_F32, torch.bfloat16: KVQ_BF16, torch.float16: KVQ_F16}
 
@@ -49,6 +50,8 @@ class KvqCacheDesc(ctypes.Structure):
         ("group_v", ctypes.c_int32), ("reserved", ctypes.c_int32),
         ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
         ("k_params", ctypes.c_void_p), ("v_params", ctypes.c_void_p),
+        ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+        ("block_table", ctypes.c_void_p),
     ]
 
 
@@ -132,25 +135,47 @@ class KVCache:
     v_params: torch.Tensor
     rotate_keys: bool = False  # KVQ_FLAG_ROTATE_KEYS: keys stored as H k
     group_v: int = 0           # values' group size (0: same as group)
+    # KVQ_FLAG_PAGED: a pool of num_pages pages of page_size positions and an
+    # int32 block table [batch][capacity / page_size] (device); 0 / None: slots
+    page_size: int = 0
+    num_pages: int = 0
+    block_table: Optional[torch.Tensor] = None
 
     @classmethod
     def allocate(cls, batch, kv_heads, head_dim, capacity, bits_k, bits_v, group,
-                 device="cuda", rotate_keys: bool = False, group_v: int = 0) -> "KVCache":
+                 device="cuda", rotate_keys: bool = False, group_v: int = 0,
+                 page_size: int = 0, num_pages: int = 0,
+                 block_table: Optional[torch.Tensor] = None) -> "KVCache":
+        """Zeroed buffers.  With page_size > 0 the cache is paged: a pool of
+        num_pages pages and the given block table (int32 [batch][capacity /
+        page_size], moved to `device`)."""
         gv = group_v or group
-        sizes = [kvq_cache_bytes(batch, kv_heads, head_dim, capacity, bits_k, bits_v,
+        rows, length = (num_pages, page_size) if page_size else (batch, capacity)
+        sizes = [kvq_cache_bytes(rows, kv_heads, head_dim, length, bits_k, bits_v,
                                  gv if w == KVQ_V_PARAMS else group, w) for w in range(4)]
         if 0 in sizes:
             raise KvqError(KVQ_ERR_INVALID_ARG, "KVCache.allocate")
+        if page_size:
+            if block_table is None or capacity % page_size:
+                raise KvqError(KVQ_ERR_INVALID_ARG, "KVCache.allocate (paged)")
+            block_table = block_table.to(device=device, dtype=torch.int32).contiguous()
+            if tuple(block_table.shape) != (batch, capacity // page_size):
+                raise KvqError(KVQ_ERR_INVALID_ARG, "KVCache.allocate (block table shape)")
         bufs = [torch.zeros(n, dtype=torch.uint8, device=device) for n in sizes]
         return cls(batch, kv_heads, head_dim, capacity, bits_k, bits_v, group, *bufs,
-                   rotate_keys=rotate_keys, group_v=group_v)
+                   rotate_keys=rotate_keys, group_v=group_v, page_size=page_size,
+                   num_pages=num_pages if page_size else 0,
+                   block_table=block_table if page_size else None)
 
     def desc(self) -> KvqCacheDesc:
+        flags = (KVQ_FLAG_ROTATE_KEYS if self.rotate_keys else 0) | \
+            (KVQ_FLAG_PAGED if self.page_size else 0)
+        bt = _dev_ptr(self.block_table, "block_table") if self.block_table is not None else None
         return KvqCacheDesc(self.batch, self.kv_heads, self.head_dim, self.capacity,
-                            self.bits_k, self.bits_v, self.group,
-                            KVQ_FLAG_ROTATE_KEYS if self.rotate_keys else 0, self.group_v, 0,
+                            self.bits_k, self.bits_v, self.group, flags, self.group_v, 0,
                             _dev_ptr(self.k_codes, "k_codes"), _dev_ptr(self.v_codes, "v_codes"),
-                            _dev_ptr(self.k_params, "k_params"), _dev_ptr(self.v_params, "v_params"))
+                            _dev_ptr(self.k_params, "k_params"), _dev_ptr(self.v_params, "v_params"),
+                            self.page_size, self.num_pages, bt)
 
 
 def kvq_validate_cache(cache: KVCache) -> int:

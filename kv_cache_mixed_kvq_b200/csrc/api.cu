@@ -66,7 +66,7 @@ int check_shape(int B, int Hkv, int D, int cap, int bk, int bv, int G) {
 int group_v_of(const kvq_cache_desc* c) { return c->group_v != 0 ? c->group_v : c->group; }
 
 int check_cache(const kvq_cache_desc* c) {
-  if (!c || (c->flags & ~KVQ_FLAG_ROTATE_KEYS) != 0 || c->reserved != 0)
+  if (!c || (c->flags & ~(KVQ_FLAG_ROTATE_KEYS | KVQ_FLAG_PAGED)) != 0 || c->reserved != 0)
     return KVQ_ERR_INVALID_ARG;
   int st = check_shape(c->batch, c->kv_heads, c->head_dim, c->capacity, c->bits_k, c->bits_v,
                        c->group);
@@ -79,7 +79,29 @@ int check_cache(const kvq_cache_desc* c) {
   const void* ptrs[4] = {c->k_codes, c->v_codes, c->k_params, c->v_params};
   for (const void* p : ptrs)
     if (!p || !aligned(p, 16)) return KVQ_ERR_INVALID_ARG;
+  if (c->flags & KVQ_FLAG_PAGED) {
+    // pages of a power-of-two number of positions, at least one decode
+    // stage (32 positions) so that no copy crosses a page
+    const int P = c->page_size;
+    if (P < 32 || (P & (P - 1)) != 0 || c->capacity % P != 0 || c->num_pages < 1 ||
+        !c->block_table || !aligned(c->block_table, 4))
+      return KVQ_ERR_INVALID_ARG;
+  } else if (c->page_size != 0 || c->num_pages != 0 || c->block_table) {
+    return KVQ_ERR_INVALID_ARG;
+  }
   return KVQ_OK;
+}
+
+// Page mapping of a cache (block_table NULL: slot layout).
+void page_args(const kvq_cache_desc* c, const int32_t** table, int* shift, int* per_seq,
+               int* num_pages) {
+  const bool paged = (c->flags & KVQ_FLAG_PAGED) != 0;
+  *table = paged ? c->block_table : nullptr;
+  int sh = 0;
+  while (paged && (1 << sh) < c->page_size) ++sh;
+  *shift = sh;
+  *per_seq = paged ? c->capacity >> sh : 0;
+  *num_pages = paged ? c->num_pages : 0;
 }
 
 bool valid_dtype(int t) { return t == KVQ_F32 || t == KVQ_BF16 || t == KVQ_F16; }
@@ -277,6 +299,7 @@ int kvq_quantize_append(const kvq_cache_desc* cache, const void* k, const void* 
   a.group = cache->group;
   a.group_v = group_v_of(cache);
   a.rotate_keys = (cache->flags & KVQ_FLAG_ROTATE_KEYS) != 0;
+  page_args(cache, &a.block_table, &a.page_shift, &a.pages_per_seq, &a.num_pages);
   st = error_word(&a.err);
   if (st != KVQ_OK) return st;
   return to_status(kvq::launch_quantize_append(a, reinterpret_cast<cudaStream_t>(stream)));
@@ -345,6 +368,7 @@ int kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int32_t q_d
     a.num_splits = p.num_splits;
     a.sm_scale_log2 = scale * 1.4426950408889634f;
     a.rotate_q = (cache->flags & KVQ_FLAG_ROTATE_KEYS) != 0;
+    page_args(cache, &a.block_table, &a.page_shift, &a.pages_per_seq, &a.num_pages);
     a.ws_o = ws_o;
     a.ws_lse = ws_lse;
     a.direct = p.direct;

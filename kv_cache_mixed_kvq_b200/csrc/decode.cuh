@@ -257,27 +257,47 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   const int my_first = warp * 16 * C::TPW;
   const int my_iters = n_tok > my_first ? (n_tok - my_first + C::kStageTokens - 1) / C::kStageTokens : 0;
   uint8_t* wring = smem + warp * C::kSlots * C::SLOT_BYTES;
-  const uint8_t* kb = a.k_codes + slot * a.capacity * C::KROW;
-  const uint8_t* vb = a.v_codes + slot * (a.capacity / 16) * C::VTILE;
-  const uint8_t* kpb = reinterpret_cast<const uint8_t*>(a.k_params) + slot * a.capacity * C::PROWK;
-  const uint8_t* vpb = reinterpret_cast<const uint8_t*>(a.v_params) + slot * a.capacity * C::PROWV;
-  auto issue = [&](int it, int sl) {
+  // A stage's 16*TPW positions start at a multiple of 16*TPW, so they never
+  // span two pages of the paged layout (pages hold a power of two >= 32).
+  static_assert(32 % (16 * C::TPW) == 0, "a stage must fit in the smallest page");
+  // Row index (positions of K rows and parameters) of position tb of this
+  // slot; in the paged layout the row inside (page, kv head), or -1 when the
+  // block table names no page of the pool.
+  auto row_of = [&](int tb) -> long long {
+    if (a.block_table == nullptr) return static_cast<long long>(slot) * a.capacity + tb;
+    const int j = tb >> a.page_shift;
+    const int page = a.block_table[static_cast<size_t>(b) * a.pages_per_seq + j];
+    if (page < 0 || page >= a.num_pages) return -1;
+    return ((static_cast<long long>(page) * a.kv_heads + hk) << a.page_shift) +
+           (tb - (j << a.page_shift));
+  };
+  auto issue = [&](int it, int sl, long long row) {
     const int base = it * C::kStageTokens + my_first;  // multiple of 16
     const int n16 = (min(16 * C::TPW, n_tok - base) + 15) & ~15;
-    const int tb = t0 + base;
     uint8_t* dst = wring + sl * C::SLOT_BYTES;
+    if (row < 0) {
+      // no page: nothing is read (the row's output is unspecified); the
+      // stage completes at once so that the pipeline keeps going
+      flag_error(a.err, KVQ_DEVERR_BAD_PAGE);
+      mbar_arrive_expect_tx(&wfull[sl], 0);
+      return;
+    }
     const uint32_t kbytes = n16 * C::KROW, vbytes = (n16 / 16) * C::VTILE;
     const uint32_t pkbytes = n16 * C::PROWK, pvbytes = n16 * C::PROWV;
+    const size_t r = static_cast<size_t>(row);
     mbar_arrive_expect_tx(&wfull[sl], kbytes + vbytes + pkbytes + pvbytes);
-    bulk_copy_g2s(dst, kb + static_cast<size_t>(tb) * C::KROW, kbytes, &wfull[sl]);
-    bulk_copy_g2s(dst + C::SLOT_K, vb + static_cast<size_t>(tb / 16) * C::VTILE, vbytes, &wfull[sl]);
-    bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V, kpb + static_cast<size_t>(tb) * C::PROWK, pkbytes,
+    bulk_copy_g2s(dst, a.k_codes + r * C::KROW, kbytes, &wfull[sl]);
+    bulk_copy_g2s(dst + C::SLOT_K, a.v_codes + (r / 16) * C::VTILE, vbytes, &wfull[sl]);
+    bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V,
+                  reinterpret_cast<const uint8_t*>(a.k_params) + r * C::PROWK, pkbytes,
                   &wfull[sl]);
     bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V + C::SLOT_PK,
-                  vpb + static_cast<size_t>(tb) * C::PROWV, pvbytes, &wfull[sl]);
+                  reinterpret_cast<const uint8_t*>(a.v_params) + r * C::PROWV, pvbytes,
+                  &wfull[sl]);
   };
+  auto stage_row = [&](int it) { return row_of(t0 + it * C::kStageTokens + my_first); };
   if (lane == 0)
-    for (int it = 0; it < min(C::kSlots, my_iters); ++it) issue(it, it);
+    for (int it = 0; it < min(C::kSlots, my_iters); ++it) issue(it, it, stage_row(it));
   __syncwarp();
 
   // ------------------------------------------------------------ consumers
@@ -720,6 +740,10 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     uint32_t phase = 0;
     int it = 0;
     for (; it < my_iters; ++it) {
+      // row of the stage this slot is refilled with, looked up before the
+      // arithmetic so that a block-table read overlaps it
+      const long long next_row =
+          (lane == 0 && it + C::kSlots < my_iters) ? stage_row(it + C::kSlots) : 0;
       if (!mbar_wait_bounded(&wfull[sl], phase, err)) break;
       const uint8_t* st = wring + sl * C::SLOT_BYTES;
       const int base = it * C::kStageTokens + my_first;  // first position of this slot
@@ -740,7 +764,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         // the warp's reads of this slot are done (registers); hand it back to
         // the copy engine for a later stage
         fence_proxy_async_shared();
-        issue(it + C::kSlots, sl);
+        issue(it + C::kSlots, sl, next_row);
       }
       if (++sl == C::kSlots) {
         sl = 0;

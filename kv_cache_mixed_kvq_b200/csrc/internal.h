@@ -42,6 +42,12 @@ struct QuantizeArgs {
   int group_v;       // values' group size
   uint32_t* err;
   bool rotate_keys;  // store keys as H k (Walsh-Hadamard along head_dim)
+  // Paged layout (block_table != NULL): position p of batch row b is local
+  // position p mod 2^page_shift of page block_table[b * pages_per_seq +
+  // (p >> page_shift)]; (page, kv head) is laid out like a slot of
+  // 2^page_shift positions.
+  const int32_t* block_table;
+  int page_shift, pages_per_seq, num_pages;
 };
 
 cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream);
@@ -62,6 +68,8 @@ struct DecodeArgs {
   int num_splits;     // grid.x
   float sm_scale_log2;  // softmax scale times log2(e)
   bool rotate_q;        // keys are stored rotated: use H q / D
+  const int32_t* block_table;  // paged layout, as in QuantizeArgs (NULL: slots)
+  int page_shift, pages_per_seq, num_pages;
   float* ws_o;        // [B][Hq][num_splits][D] partial outputs
   float* ws_lse;      // [B][Hq][num_splits] log2-domain log-sum-exp
   uint32_t* err;

@@ -29,6 +29,9 @@
 // A tile fully covered by the append is assembled in shared memory and
 // written with 16-byte stores; a tile at the edge of the appended range is
 // written element by element so that positions outside it stay untouched.
+// In the paged layout a tile (16 positions) never spans two pages; its page
+// comes from the block table and its rows and V tile are addressed inside
+// (page, kv head) exactly as inside a slot.
 #pragma once
 
 #include "common.cuh"
@@ -264,6 +267,24 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
   if (tile * 16 >= end) return;
   const bool full_tile = tile * 16 >= pos && tile * 16 + 16 <= end;
   const size_t slot = static_cast<size_t>(b) * a.kv_heads + h;
+  // destination: row index of the tile's first position in the per-position
+  // arrays (K rows, parameters) and index of its V tile
+  size_t row0, vt;
+  if (a.block_table == nullptr) {
+    row0 = slot * a.capacity + tile * 16;
+    vt = slot * (a.capacity / 16) + tile;
+  } else {
+    const int j = (tile * 16) >> a.page_shift;
+    const int page = a.block_table[static_cast<size_t>(b) * a.pages_per_seq + j];
+    if (page < 0 || page >= a.num_pages) {
+      if (threadIdx.x == 0) flag_error(a.err, KVQ_DEVERR_BAD_PAGE);
+      return;
+    }
+    const size_t vslot = static_cast<size_t>(page) * a.kv_heads + h;
+    const int local = tile * 16 - (j << a.page_shift);
+    row0 = (vslot << a.page_shift) + local;
+    vt = (vslot << (a.page_shift - 4)) + local / 16;
+  }
 
   const int t = threadIdx.x;
   const bool is_v = t >= C::KT;  // warp-uniform
@@ -311,7 +332,7 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
 #pragma unroll
         for (int q = 0; q < NPAR; ++q) skp[k * NGK + first_group + q] = par[q];
     } else if (valid) {
-      uint8_t* row = a.k_codes + (slot * a.capacity + p) * C::KROW;
+      uint8_t* row = a.k_codes + (row0 + k) * C::KROW;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
         *reinterpret_cast<uint32_t*>(row + c * C::KSLICE + 4 * w) =
@@ -319,7 +340,7 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
       if (reports)
 #pragma unroll
         for (int q = 0; q < NPAR; ++q)
-          a.k_params[(slot * a.capacity + p) * NGK + first_group + q] = par[q];
+          a.k_params[(row0 + k) * NGK + first_group + q] = par[q];
     }
   } else {
     // ---------------------------------------------------------- values
@@ -352,23 +373,23 @@ __global__ void __launch_bounds__(C::THREADS) quantize_append_kernel(const Quant
 #pragma unroll
         for (int q = 0; q < NPAR; ++q) svp[k * NGV + first_group + q] = par[q];
     } else if (valid) {
-      uint8_t* gt = a.v_codes + (slot * (a.capacity / 16) + tile) * C::VTILE;
+      uint8_t* gt = a.v_codes + vt * C::VTILE;
 #pragma unroll
       for (int g = 0; g < 8; ++g)
         *reinterpret_cast<uint16_t*>(gt + off0 + 4 * g * C::VP) = static_cast<uint16_t>(acc[g]);
       if (reports)
 #pragma unroll
         for (int q = 0; q < NPAR; ++q)
-          a.v_params[(slot * a.capacity + p) * NGV + first_group + q] = par[q];
+          a.v_params[(row0 + k) * NGV + first_group + q] = par[q];
     }
   }
 
   if (full_tile) {
     __syncthreads();
-    uint4* gk = reinterpret_cast<uint4*>(a.k_codes + (slot * a.capacity + tile * 16) * C::KROW);
-    uint4* gv = reinterpret_cast<uint4*>(a.v_codes + (slot * (a.capacity / 16) + tile) * C::VTILE);
-    uint4* gkp = reinterpret_cast<uint4*>(a.k_params + (slot * a.capacity + tile * 16) * NGK);
-    uint4* gvp = reinterpret_cast<uint4*>(a.v_params + (slot * a.capacity + tile * 16) * NGV);
+    uint4* gk = reinterpret_cast<uint4*>(a.k_codes + row0 * C::KROW);
+    uint4* gv = reinterpret_cast<uint4*>(a.v_codes + vt * C::VTILE);
+    uint4* gkp = reinterpret_cast<uint4*>(a.k_params + row0 * NGK);
+    uint4* gvp = reinterpret_cast<uint4*>(a.v_params + row0 * NGV);
     for (int i = t; i < 16 * C::KROW / 16; i += C::THREADS) gk[i] = reinterpret_cast<const uint4*>(sk)[i];
     for (int i = t; i < C::VTILE / 16; i += C::THREADS) gv[i] = reinterpret_cast<const uint4*>(sv)[i];
     for (int i = t; i < NGK * 4; i += C::THREADS)  // 16 * NGK words = 4 * NGK uint4

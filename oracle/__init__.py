@@ -250,6 +250,11 @@ class PagedHostCache:
         p = self.pool
         return [p.k_codes, p.v_codes, p.k_params, p.v_params]
 
+    k_codes = property(lambda self: self.pool.k_codes)
+    v_codes = property(lambda self: self.pool.v_codes)
+    k_params = property(lambda self: self.pool.k_params)
+    v_params = property(lambda self: self.pool.v_params)
+
     def _row_cache(self, rows: int) -> HostCache:
         D, bk, bv, g, rot, gv = self.shape
         return HostCache(rows, self.Hkv, D, self.cap, bk, bv, g, rotate_keys=rot, group_v=gv)

@@ -55,7 +55,8 @@ def test_cache_bytes_rejects_bad_shapes(args):
 
 def _desc(**kw):
     d = dict(batch=1, kv_heads=2, head_dim=128, capacity=64, bits_k=4, bits_v=2, group=64,
-             flags=0, group_v=0, reserved=0, k_codes=0x1000, v_codes=0x2000, k_params=0x3000, v_params=0x4000)
+             flags=0, group_v=0, reserved=0, k_codes=0x1000, v_codes=0x2000, k_params=0x3000, v_params=0x4000,
+             page_size=0, num_pages=0, block_table=None)
     d.update(kw)
     return kvq.KvqCacheDesc(*d.values())
 
@@ -66,7 +67,20 @@ def test_validate_cache_host_only():
     assert lib.kvq_validate_cache(ctypes.byref(_desc(k_codes=0x1008))) == kvq.KVQ_ERR_INVALID_ARG
     assert lib.kvq_validate_cache(ctypes.byref(_desc(v_params=0))) == kvq.KVQ_ERR_INVALID_ARG
     assert lib.kvq_validate_cache(ctypes.byref(_desc(flags=kvq.KVQ_FLAG_ROTATE_KEYS))) == kvq.KVQ_OK
-    assert lib.kvq_validate_cache(ctypes.byref(_desc(flags=2))) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_validate_cache(ctypes.byref(_desc(flags=4))) == kvq.KVQ_ERR_INVALID_ARG
+    # paged layout: power-of-two pages of >= 32 positions dividing capacity,
+    # a pool of >= 1 page and an aligned block table; none of it without the flag
+    paged = dict(flags=kvq.KVQ_FLAG_PAGED, page_size=32, num_pages=5, block_table=0x5000)
+    assert lib.kvq_validate_cache(ctypes.byref(_desc(**paged))) == kvq.KVQ_OK
+    assert lib.kvq_validate_cache(ctypes.byref(_desc(**dict(paged, page_size=64)))) == kvq.KVQ_OK
+    assert lib.kvq_validate_cache(ctypes.byref(
+        _desc(**dict(paged, flags=3)))) == kvq.KVQ_OK  # with key rotation
+    for bad in (dict(page_size=16), dict(page_size=48), dict(page_size=128), dict(page_size=0),
+                dict(num_pages=0), dict(block_table=None), dict(block_table=0x5002)):
+        assert lib.kvq_validate_cache(ctypes.byref(_desc(**dict(paged, **bad)))) == \
+            kvq.KVQ_ERR_INVALID_ARG, bad
+    for stray in (dict(page_size=32), dict(num_pages=1), dict(block_table=0x5000)):
+        assert lib.kvq_validate_cache(ctypes.byref(_desc(**stray))) == kvq.KVQ_ERR_INVALID_ARG
     assert lib.kvq_validate_cache(ctypes.byref(_desc(reserved=1))) == kvq.KVQ_ERR_INVALID_ARG
     # value groups: equal or coarser than the keys' (group 64 here)
     assert lib.kvq_validate_cache(ctypes.byref(_desc(group_v=128))) == kvq.KVQ_OK
