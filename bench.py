@@ -193,6 +193,8 @@ class Arm:
         self.pos_t = torch.tensor(self.pos, dtype=torch.int32, device=device)
         self.sets = []
         self.page_size = page_size
+        if page_size:  # the logical capacity of a paged cache is whole pages
+            self.cap = -(-self.cap // page_size) * page_size
         for r in range(rotate):
             paged = {}
             if page_size:

@@ -260,31 +260,33 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   // A stage's 16*TPW positions start at a multiple of 16*TPW, so they never
   // span two pages of the paged layout (pages hold a power of two >= 32).
   static_assert(32 % (16 * C::TPW) == 0, "a stage must fit in the smallest page");
-  // Row index (positions of K rows and parameters) of position tb of this
-  // slot; in the paged layout the row inside (page, kv head), or -1 when the
-  // block table names no page of the pool.
-  auto row_of = [&](int tb) -> long long {
-    if (a.block_table == nullptr) return static_cast<long long>(slot) * a.capacity + tb;
-    const int j = tb >> a.page_shift;
-    const int page = a.block_table[static_cast<size_t>(b) * a.pages_per_seq + j];
-    if (page < 0 || page >= a.num_pages) return -1;
-    return ((static_cast<long long>(page) * a.kv_heads + hk) << a.page_shift) +
-           (tb - (j << a.page_shift));
+  // Position tb of this slot (the first of a stage).  Slot layout: row
+  // slot * capacity + tb of the per-position arrays.  Paged layout: its page
+  // (block-table entry, looked up ahead by page_of) and the row inside
+  // (page, kv head); a page outside the pool is never read.
+  auto page_of = [&](int it) -> int {
+    const int tb = t0 + it * C::kStageTokens + my_first;
+    return a.block_table[static_cast<size_t>(b) * a.pages_per_seq + (tb >> a.page_shift)];
   };
-  auto issue = [&](int it, int sl, long long row) {
+  auto issue = [&](int it, int sl, int page) {
     const int base = it * C::kStageTokens + my_first;  // multiple of 16
     const int n16 = (min(16 * C::TPW, n_tok - base) + 15) & ~15;
+    const int tb = t0 + base;
     uint8_t* dst = wring + sl * C::SLOT_BYTES;
-    if (row < 0) {
-      // no page: nothing is read (the row's output is unspecified); the
-      // stage completes at once so that the pipeline keeps going
-      flag_error(a.err, KVQ_DEVERR_BAD_PAGE);
-      mbar_arrive_expect_tx(&wfull[sl], 0);
-      return;
+    size_t r = slot * a.capacity + tb;
+    if (a.block_table != nullptr) {
+      if (page < 0 || page >= a.num_pages) {
+        // no page: nothing is read (the row's output is unspecified); the
+        // stage completes at once so that the pipeline keeps going
+        flag_error(a.err, KVQ_DEVERR_BAD_PAGE);
+        mbar_arrive_expect_tx(&wfull[sl], 0);
+        return;
+      }
+      const int local = tb & ((1 << a.page_shift) - 1);
+      r = ((static_cast<size_t>(page) * a.kv_heads + hk) << a.page_shift) + local;
     }
     const uint32_t kbytes = n16 * C::KROW, vbytes = (n16 / 16) * C::VTILE;
     const uint32_t pkbytes = n16 * C::PROWK, pvbytes = n16 * C::PROWV;
-    const size_t r = static_cast<size_t>(row);
     mbar_arrive_expect_tx(&wfull[sl], kbytes + vbytes + pkbytes + pvbytes);
     bulk_copy_g2s(dst, a.k_codes + r * C::KROW, kbytes, &wfull[sl]);
     bulk_copy_g2s(dst + C::SLOT_K, a.v_codes + (r / 16) * C::VTILE, vbytes, &wfull[sl]);
@@ -295,9 +297,9 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
                   reinterpret_cast<const uint8_t*>(a.v_params) + r * C::PROWV, pvbytes,
                   &wfull[sl]);
   };
-  auto stage_row = [&](int it) { return row_of(t0 + it * C::kStageTokens + my_first); };
   if (lane == 0)
-    for (int it = 0; it < min(C::kSlots, my_iters); ++it) issue(it, it, stage_row(it));
+    for (int it = 0; it < min(C::kSlots, my_iters); ++it)
+      issue(it, it, a.block_table != nullptr ? page_of(it) : 0);
   __syncwarp();
 
   // ------------------------------------------------------------ consumers
@@ -740,10 +742,12 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     uint32_t phase = 0;
     int it = 0;
     for (; it < my_iters; ++it) {
-      // row of the stage this slot is refilled with, looked up before the
-      // arithmetic so that a block-table read overlaps it
-      const long long next_row =
-          (lane == 0 && it + C::kSlots < my_iters) ? stage_row(it + C::kSlots) : 0;
+      // paged layout: the page of the stage this slot is refilled with,
+      // looked up before the arithmetic so that the block-table read
+      // overlaps it
+      int next_page = 0;
+      if (a.block_table != nullptr && lane == 0 && it + C::kSlots < my_iters)
+        next_page = page_of(it + C::kSlots);
       if (!mbar_wait_bounded(&wfull[sl], phase, err)) break;
       const uint8_t* st = wring + sl * C::SLOT_BYTES;
       const int base = it * C::kStageTokens + my_first;  // first position of this slot
@@ -764,7 +768,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         // the warp's reads of this slot are done (registers); hand it back to
         // the copy engine for a later stage
         fence_proxy_async_shared();
-        issue(it + C::kSlots, sl, next_row);
+        issue(it + C::kSlots, sl, next_page);
       }
       if (++sl == C::kSlots) {
         sl = 0;
