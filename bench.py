@@ -182,7 +182,7 @@ class Arm:
     """Device buffers for R rotating sets of inputs + caches, and the step."""
 
     def __init__(self, w, bits, rotate: int, device, rotate_keys: bool = False,
-                 group_v: int = 0, page_size: int = 0):
+                 group_v: int = 0, page_size: int = 0, fused: bool = False):
         import kv_cache_mixed_kvq_b200 as kvq
         self.kvq = kvq
         self.w, self.bits = w, bits
@@ -193,6 +193,8 @@ class Arm:
         self.pos_t = torch.tensor(self.pos, dtype=torch.int32, device=device)
         self.sets = []
         self.page_size = page_size
+        # fused: the step's append runs inside the decode call (one launch)
+        self.fused = bool(fused) and self.n_new > 0
         if page_size:  # the logical capacity of a paged cache is whole pages
             self.cap = -(-self.cap // page_size) * page_size
         for r in range(rotate):
@@ -227,20 +229,25 @@ class Arm:
 
     def quantize(self, r):
         s = self.sets[r]
-        if self.n_new:
+        if self.n_new and not self.fused:
             self.kvq.kvq_quantize_append(s["cache"], s["k"], s["v"], self.pos_t)
 
     def decode(self, r):
         s = self.sets[r]
-        self.kvq.kvq_decode_attention(s["cache"], s["q"], self.lens, self.max_len, out=s["out"],
-                                      workspace=self.ws)
+        if self.fused:
+            self.kvq.kvq_append_decode_attention(s["cache"], s["k"], s["v"], s["q"], self.lens,
+                                                 self.max_len, out=s["out"], workspace=self.ws)
+        else:
+            self.kvq.kvq_decode_attention(s["cache"], s["q"], self.lens, self.max_len,
+                                          out=s["out"], workspace=self.ws)
 
     def step(self, r):
         self.quantize(r)
         self.decode(r)
 
     launches_per_step = property(
-        lambda self: (1 if self.n_new else 0) + (1 if self.num_splits == 1 else 2))
+        lambda self: (1 if self.n_new and not self.fused else 0) +
+        (1 if self.num_splits == 1 else 2))
 
 
 def _slot_view(cache, b):
@@ -267,7 +274,7 @@ def run_ours(args, rank, world, device):
         if w.name == "long" else w.bits[0]
     rotate = args.rotate
     arm = Arm(w, bits, rotate, device, rotate_keys=args.rotate_keys, group_v=args.group_v,
-              page_size=args.page_size)
+              page_size=args.page_size, fused=args.fused)
     stream = torch.cuda.current_stream()
 
     # warm-up (also loads every kernel and the error-word address)
@@ -320,14 +327,16 @@ def run_ours(args, rank, world, device):
         if name not in kern:
             continue
         t_s = kern[name] / 1e3
-        ach = nbytes[key] / t_s / 1e9
+        # the fused call also moves the append's bytes
+        kbytes = nbytes[key] + (nbytes["quantize"] if arm.fused and key == "decode" else 0)
+        ach = kbytes / t_s / 1e9
         roof[name] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak,
                       "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
                       "traffic": measured_traffic(
                           (["quantize_rot"] if args.rotate_keys else ["quantize"])
                           if key == "quantize" else
                           (["decode"] if arm.num_splits == 1 else ["decode", "combine"]), w.name),
-                      "ms": round(kern[name], 5), "algorithmic_bytes": nbytes[key],
+                      "ms": round(kern[name], 5), "algorithmic_bytes": kbytes,
                       "peak_source": f"{peak_kind} hbm_gbs (copy)"}
     dominant = "quantize" if "quantize" in roof and kern["quantize"] >= kern.get(
         "decode_attention", 0) else "decode_attention"
@@ -354,7 +363,9 @@ def run_ours(args, rank, world, device):
             "rotate_keys": bool(args.rotate_keys),
             "group_v": args.group_v or w.group,
             "page_size": args.page_size,
+            "fused_append": arm.fused,
             "step": ("quantize full cache + decode + combine" if w.name == "llama3_8b" else
+                     f"append {arm.n_new} inside the decode + combine" if arm.fused else
                      f"append {arm.n_new} + decode + combine"),
             "split_tokens": arm.split_tokens,
             "l2": f"{rotate} rotating input/cache sets (each step's data last touched "
@@ -426,7 +437,7 @@ def per_kernel_times(arm, rotate, stream, reps):
         q.append(e[0].elapsed_time(e[1]))
         d.append(e[1].elapsed_time(e[2]))
     out = {"decode_attention": statistics.mean(d)}
-    if arm.n_new:
+    if arm.n_new and not arm.fused:
         out["quantize"] = statistics.mean(q)
     return out
 
@@ -447,10 +458,14 @@ def run_e2e(arm, args, step_bytes, world, device):
         k_dev.copy_(hk, non_blocking=True)
         v_dev.copy_(hv, non_blocking=True)
         q_dev.copy_(hq, non_blocking=True)
-        if arm.n_new:
-            arm.kvq.kvq_quantize_append(cache, k_dev, v_dev, arm.pos_t)
-        arm.kvq.kvq_decode_attention(cache, q_dev, arm.lens, arm.max_len, out=s0["out"],
-                                     workspace=arm.ws)
+        if arm.fused:
+            arm.kvq.kvq_append_decode_attention(cache, k_dev, v_dev, q_dev, arm.lens,
+                                                arm.max_len, out=s0["out"], workspace=arm.ws)
+        else:
+            if arm.n_new:
+                arm.kvq.kvq_quantize_append(cache, k_dev, v_dev, arm.pos_t)
+            arm.kvq.kvq_decode_attention(cache, q_dev, arm.lens, arm.max_len, out=s0["out"],
+                                         workspace=arm.ws)
         hout.copy_(s0["out"], non_blocking=True)
 
     for _ in range(args.warmup):
@@ -556,6 +571,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--group-v", type=int, default=0,
                     help="values' group size (default: the workload's group)")
+    ap.add_argument("--fused", action="store_true",
+                    help="append inside the decode call (kvq_append_decode_attention)")
     ap.add_argument("--page-size", type=int, default=0,
                     help="paged cache layout with pages of this many positions (0: slots)")
     ap.add_argument("--rotate-keys", action="store_true",

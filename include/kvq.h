@@ -243,7 +243,9 @@ int kvq_validate_cache(const kvq_cache_desc* cache);
  * with bits_v, in the format above.  Positions outside the new range are not
  * touched (the other half of a shared V word is preserved).  Rows whose
  * range would pass `capacity` (or with pos[b] < 0) are skipped and flag
- * KVQ_DEVERR_CAPACITY (KVQ_DEVERR_BAD_POS).  Does not advance any length:
+ * KVQ_DEVERR_CAPACITY (KVQ_DEVERR_BAD_POS).  Paged layout: each 16-position
+ * tile is written to the page its block-table entry names; tiles whose entry
+ * is outside [0, num_pages) are skipped and flag KVQ_DEVERR_BAD_PAGE.  Does not advance any length:
  * the caller owns seq_lens.  One kernel launch.
  */
 int kvq_quantize_append(const kvq_cache_desc* cache, const void* k,
@@ -267,7 +269,10 @@ size_t kvq_decode_workspace_bytes(const kvq_cache_desc* cache,
  *                 head hq reads kv head hq / (Hq / Hkv)).
  *   seq_lens    : device int32[B]; batch row b attends to positions
  *                 [0, seq_lens[b]).  Values above max_seq_len or capacity
- *                 are clamped and flag KVQ_DEVERR_SEQ_LEN.
+ *                 are clamped and flag KVQ_DEVERR_SEQ_LEN.  Paged layout:
+ *                 positions are read through the block table; a row that
+ *                 reaches an entry outside the pool flags
+ *                 KVQ_DEVERR_BAD_PAGE and its output is unspecified.
  *   max_seq_len : host upper bound of seq_lens (sizes the split-K grid).
  *   sm_scale    : softmax scale; <= 0 selects 1/sqrt(D).
  *   out         : device, [B][Hq][D], out_dtype in {F32, BF16, F16}.
@@ -287,6 +292,36 @@ int kvq_decode_attention(const kvq_cache_desc* cache, const void* q,
                          float sm_scale, void* out, int32_t out_dtype,
                          void* workspace, size_t workspace_bytes,
                          kvq_stream_t stream);
+
+/*
+ * Decode attention with the step's append fused in (one launch, plus the
+ * combine when rows are split): the same result as
+ *   kvq_quantize_append(cache, k_new, v_new, in_dtype, pos, n_new, stream)
+ *   kvq_decode_attention(cache, q, ..., seq_lens, ...)
+ * with pos[b] = seq_lens[b] - n_new, i.e. the n_new new tokens of every batch
+ * row are the last ones it attends to (a decode step that appends its own
+ * key and value rows).  The split-K CTA that owns a new position quantizes
+ * and writes it before reading it ("Quantize What Counts", summary page,
+ * "Problem statement": the cache is written once per token and read by
+ * every later step).
+ *
+ *   k_new, v_new : device, [B][Hkv][n_new][D] row-major, in_dtype (F32, BF16
+ *                  or F16), 16-byte aligned.  n_new = 0: plain decode.
+ *   other arguments as for kvq_decode_attention(); the workspace size is the
+ *   same (kvq_decode_workspace_bytes()).
+ *
+ * Rows with seq_lens[b] < n_new append nothing and flag KVQ_DEVERR_BAD_POS;
+ * rows whose length is clamped (KVQ_DEVERR_SEQ_LEN) append nothing.  The
+ * written bytes equal those of kvq_quantize_append() (same quantizer, same
+ * format; positions outside the new range keep their bytes).
+ */
+int kvq_append_decode_attention(const kvq_cache_desc* cache, const void* k_new,
+                                const void* v_new, int32_t in_dtype, int32_t n_new,
+                                const void* q, int32_t q_dtype, int32_t num_q_heads,
+                                const int32_t* seq_lens, int32_t max_seq_len,
+                                float sm_scale, void* out, int32_t out_dtype,
+                                void* workspace, size_t workspace_bytes,
+                                kvq_stream_t stream);
 
 /*
  * Size of the fixed device scratch array used by

@@ -81,6 +81,9 @@ def library() -> ctypes.CDLL:
     lib.kvq_decode_split_tokens.restype = I32
     lib.kvq_decode_attention.argtypes = [D, P, I32, I32, P, I32, ctypes.c_float, P, I32, P, SZ, P]
     lib.kvq_decode_attention.restype = ctypes.c_int
+    lib.kvq_append_decode_attention.argtypes = [D, P, P, I32, I32, P, I32, I32, P, I32,
+                                                ctypes.c_float, P, I32, P, SZ, P]
+    lib.kvq_append_decode_attention.restype = ctypes.c_int
     lib.kvq_device_error_flags.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
     lib.kvq_device_error_flags.restype = ctypes.c_int
     lib.kvq_last_device_error.argtypes = [P]
@@ -232,6 +235,38 @@ def kvq_decode_attention(cache: KVCache, q: torch.Tensor, seq_lens: torch.Tensor
                                   float(sm_scale), _dev_ptr(out, "out"), _DTYPE[out.dtype],
                                   ws_ptr, ws_bytes, _stream_ptr(stream))
     _check(st, "kvq_decode_attention")
+    return out
+
+
+def kvq_append_decode_attention(cache: KVCache, k_new: torch.Tensor, v_new: torch.Tensor,
+                                q: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,
+                                sm_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                out_dtype: Optional[torch.dtype] = None,
+                                workspace: Optional[torch.Tensor] = None,
+                                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Append k_new, v_new ([B][Hkv][n_new][D]) at positions seq_lens[b] - n_new ..
+    seq_lens[b] - 1, then attend q ([B][Hq][D]) to [0, seq_lens[b]): one fused call."""
+    if k_new.dtype != v_new.dtype or k_new.shape != v_new.shape or k_new.dim() != 4:
+        raise ValueError("k_new and v_new must be [B][Hkv][n_new][D] tensors of one dtype")
+    if q.dim() != 3:
+        raise ValueError("q must be [B][Hq][D]")
+    if seq_lens.dtype != torch.int32:
+        raise ValueError("seq_lens must be int32")
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    d = cache.desc()
+    lib = library()
+    need = int(lib.kvq_decode_workspace_bytes(ctypes.byref(d), q.shape[1], max_seq_len))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev_ptr(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.kvq_append_decode_attention(
+        ctypes.byref(d), _dev_ptr(k_new, "k_new"), _dev_ptr(v_new, "v_new"), _DTYPE[k_new.dtype],
+        k_new.shape[2], _dev_ptr(q, "q"), _DTYPE[q.dtype], q.shape[1],
+        _dev_ptr(seq_lens, "seq_lens"), int(max_seq_len), float(sm_scale), _dev_ptr(out, "out"),
+        _DTYPE[out.dtype], ws_ptr, ws_bytes, _stream_ptr(stream))
+    _check(st, "kvq_append_decode_attention")
     return out
 
 

@@ -321,10 +321,15 @@ int32_t kvq_decode_split_tokens(const kvq_cache_desc* cache, int32_t num_q_heads
   return p.split_tokens;
 }
 
-int kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int32_t q_dtype,
-                         int32_t num_q_heads, const int32_t* seq_lens, int32_t max_seq_len,
-                         float sm_scale, void* out, int32_t out_dtype, void* workspace,
-                         size_t workspace_bytes, kvq_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// Decode attention, with the step's append fused in when k_new != NULL.
+int decode_impl(const kvq_cache_desc* cache, const void* k_new, const void* v_new,
+                int32_t in_dtype, int32_t n_new, const void* q, int32_t q_dtype,
+                int32_t num_q_heads, const int32_t* seq_lens, int32_t max_seq_len,
+                float sm_scale, void* out, int32_t out_dtype, void* workspace,
+                size_t workspace_bytes, kvq_stream_t stream) {
   int st = check_decode_args(cache, num_q_heads, max_seq_len);
   if (st != KVQ_OK) return st;
   if (!valid_dtype(q_dtype) || !valid_dtype(out_dtype)) return KVQ_ERR_INVALID_ARG;
@@ -369,6 +374,10 @@ int kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int32_t q_d
     a.sm_scale_log2 = scale * 1.4426950408889634f;
     a.rotate_q = (cache->flags & KVQ_FLAG_ROTATE_KEYS) != 0;
     page_args(cache, &a.block_table, &a.page_shift, &a.pages_per_seq, &a.num_pages);
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.in_dtype = in_dtype;
+    a.n_new = n_new;
     a.ws_o = ws_o;
     a.ws_lse = ws_lse;
     a.direct = p.direct;
@@ -394,6 +403,31 @@ int kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int32_t q_d
   ca.split_tokens = p.split_tokens;
   ca.num_splits = p.num_splits;
   return to_status(kvq::launch_combine(ca, s));
+}
+}  // namespace
+
+extern "C" {
+
+int kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int32_t q_dtype,
+                         int32_t num_q_heads, const int32_t* seq_lens, int32_t max_seq_len,
+                         float sm_scale, void* out, int32_t out_dtype, void* workspace,
+                         size_t workspace_bytes, kvq_stream_t stream) {
+  return decode_impl(cache, nullptr, nullptr, 0, 0, q, q_dtype, num_q_heads, seq_lens,
+                     max_seq_len, sm_scale, out, out_dtype, workspace, workspace_bytes, stream);
+}
+
+int kvq_append_decode_attention(const kvq_cache_desc* cache, const void* k_new,
+                                const void* v_new, int32_t in_dtype, int32_t n_new,
+                                const void* q, int32_t q_dtype, int32_t num_q_heads,
+                                const int32_t* seq_lens, int32_t max_seq_len, float sm_scale,
+                                void* out, int32_t out_dtype, void* workspace,
+                                size_t workspace_bytes, kvq_stream_t stream) {
+  if (n_new < 0 || (n_new > 0 && (!valid_dtype(in_dtype) || !k_new || !v_new ||
+                                  !aligned(k_new, 16) || !aligned(v_new, 16))))
+    return KVQ_ERR_INVALID_ARG;
+  return decode_impl(cache, n_new > 0 ? k_new : nullptr, n_new > 0 ? v_new : nullptr, in_dtype,
+                     n_new, q, q_dtype, num_q_heads, seq_lens, max_seq_len, sm_scale, out,
+                     out_dtype, workspace, workspace_bytes, stream);
 }
 
 int kvq_device_error_flags(kvq_stream_t stream, uint32_t* flags) {

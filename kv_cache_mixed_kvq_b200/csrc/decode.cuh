@@ -35,6 +35,7 @@
 
 #include <type_traits>
 
+#include "append_rows.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -233,6 +234,16 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
 
   int len = a.seq_lens[b];
   const int lim = min(a.max_seq_len, a.capacity);
+  // fused append: positions [len - n_new, len) are written first; a row
+  // whose length is out of range appends nothing
+  int app_pos = -1;
+  if (a.k_new != nullptr && len <= lim) {
+    if (len < a.n_new) {
+      if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0) flag_error(a.err, KVQ_DEVERR_BAD_POS);
+    } else {
+      app_pos = len - a.n_new;
+    }
+  }
   if (len < 0 || len > lim) {
     if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0) flag_error(a.err, KVQ_DEVERR_SEQ_LEN);
     len = max(0, min(len, lim));
@@ -251,6 +262,26 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   const int t1 = min(t0 + a.split_tokens, len);
   const int n_tok = t1 - t0;
   const size_t slot = static_cast<size_t>(b) * a.kv_heads + hk;
+
+  // ---- fused append of the new positions in this split (every head-group
+  // CTA of the slot writes the same bytes), made visible to the bulk copies
+  // below before any is issued
+  if (app_pos >= 0) {
+    const int p0 = max(app_pos, t0), p1 = t1;
+    if (p0 < p1) {
+      auto row_of_pos = [&](int p) -> long long {
+        if (a.block_table == nullptr) return static_cast<long long>(slot) * a.capacity + p;
+        const int page = a.block_table[static_cast<size_t>(b) * a.pages_per_seq + (p >> a.page_shift)];
+        if (page < 0 || page >= a.num_pages) return -1;
+        return ((static_cast<long long>(page) * a.kv_heads + hk) << a.page_shift) +
+               (p & ((1 << a.page_shift) - 1));
+      };
+      append_rows<C>(a, b, hk, app_pos, p0, p1, smem + warp * 5 * D, row_of_pos);
+      fence_proxy_async_global();
+      __syncthreads();
+      fence_proxy_async_global();
+    }
+  }
 
   // ---- this warp's copy pipeline: positions [it*kStageTokens + 16*TPW*warp, +16*TPW)
   // of the split for it = 0 .. my_iters-1, kSlots copies in flight.

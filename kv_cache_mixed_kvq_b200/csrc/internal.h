@@ -70,6 +70,12 @@ struct DecodeArgs {
   bool rotate_q;        // keys are stored rotated: use H q / D
   const int32_t* block_table;  // paged layout, as in QuantizeArgs (NULL: slots)
   int page_shift, pages_per_seq, num_pages;
+  // Fused append (NULL k_new: none): before attending, each CTA quantizes
+  // the new rows k_new / v_new ([B][Hkv][n_new][D], element type in_dtype)
+  // of positions [seq_lens[b] - n_new, seq_lens[b]) that fall in its split.
+  const void* k_new;
+  const void* v_new;
+  int in_dtype, n_new;
   float* ws_o;        // [B][Hq][num_splits][D] partial outputs
   float* ws_lse;      // [B][Hq][num_splits] log2-domain log-sum-exp
   uint32_t* err;

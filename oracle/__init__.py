@@ -330,6 +330,39 @@ class PagedHostCache:
         return self.pool.dequant_row(which, page, h, p % self.P)
 
 
+def append_decode_attention(hc, k: np.ndarray, v: np.ndarray, q: np.ndarray, Hq: int, seq_lens,
+                            dtype: str | None = None, q_dtype: str | None = None,
+                            max_len: int | None = None, sm_scale: float = 0.0):
+    """Definition of the fused append + decode call, as the composition of
+    the two operations: every batch row b whose length n = seq_lens[b] is
+    within min(capacity, max_len) appends its n_new new rows at positions
+    n - n_new .. n - 1 (a row with n < n_new appends nothing and sets
+    DEVERR_BAD_POS; a row with n out of range appends nothing and the
+    decode flags it), then attention over [0, n).  `hc`: HostCache or
+    PagedHostCache.  Returns (out, flags)."""
+    n_new = k.shape[2]
+    lim = min(hc.cap, hc.cap if max_len is None else max_len)
+    lens = [int(n) for n in seq_lens]
+    flags = 0
+    # rows that append nothing get position `capacity` (past the end: the
+    # append skips them); its capacity flag is not part of this call's result
+    pos = []
+    for n in lens:
+        if n > lim:
+            pos.append(hc.cap)
+        elif n < n_new:
+            flags |= DEVERR_BAD_POS
+            pos.append(hc.cap)
+        else:
+            pos.append(n - n_new)
+    skipped = any(p == hc.cap for p in pos)
+    f = hc.quantize_append(k, v, pos, dtype=dtype)
+    flags |= (f & ~DEVERR_CAPACITY) if skipped else f
+    out, f2 = hc.decode_attention(q, Hq, lens, sm_scale=sm_scale, q_dtype=q_dtype,
+                                  max_len=max_len)
+    return out, flags | f2
+
+
 def fwht(x) -> np.ndarray:
     """Unnormalised Walsh-Hadamard transform of a binary32 vector (the oracle's
     key rotation, same butterfly order and rounding)."""

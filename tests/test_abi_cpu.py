@@ -22,7 +22,7 @@ def test_header_declares_entry_points():
     names = _declared()
     for n in ("kvq_quantize_append", "kvq_decode_attention", "kvq_cache_bytes",
               "kvq_decode_workspace_bytes", "kvq_device_error_flags", "kvq_last_device_error",
-              "kvq_decode_attention_static", "kvq_strerror"):
+              "kvq_decode_attention_static", "kvq_append_decode_attention", "kvq_strerror"):
         assert n in names
 
 
@@ -135,3 +135,20 @@ def test_strerror():
     assert kvq.kvq_strerror(kvq.KVQ_OK) == "ok"
     assert "workspace" in kvq.kvq_strerror(kvq.KVQ_ERR_WORKSPACE)
     assert kvq.kvq_strerror(99) == "unknown status"
+
+
+def test_fused_append_rejects_before_launch():
+    lib = kvq.library()
+    d = _desc()
+    f = lib.kvq_append_decode_attention
+
+    def call(k=0x500, v=0x600, dt=1, n=1, hq=8, q=0x100):
+        return f(ctypes.byref(d), k, v, dt, n, q, 1, hq, 0x200, 64, 0.0, 0x300, 1, 0x400,
+                 1 << 20, None)
+
+    assert call(n=-1) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(k=None) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(v=0x608) == kvq.KVQ_ERR_INVALID_ARG      # misaligned
+    assert call(dt=5) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(hq=7) == kvq.KVQ_ERR_INVALID_ARG         # decode checks still apply
+    assert call(q=0) == kvq.KVQ_ERR_INVALID_ARG
