@@ -135,6 +135,9 @@ cudaError_t prepare_kernel(const DecodeKernel& k) {
   std::lock_guard<std::mutex> lock(mu);
   if (done.count({dev, k.fn})) return cudaSuccess;
   e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem_bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k.fn_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             k.smem_bytes);
   if (e == cudaSuccess) done.insert({dev, k.fn});
   return e;
 }
@@ -386,7 +389,8 @@ int decode_impl(const kvq_cache_desc* cache, const void* k_new, const void* v_ne
     st = error_word(&a.err);
     if (st != KVQ_OK) return st;
     const dim3 grid(p.num_splits, cache->kv_heads * p.head_groups, cache->batch);
-    if (k.launch(a, grid, s) != cudaSuccess) return KVQ_ERR_CUDA;
+    if ((k_new != nullptr ? k.launch_fused : k.launch)(a, grid, s) != cudaSuccess)
+      return KVQ_ERR_CUDA;
     if (p.direct) return KVQ_OK;
   }
   kvq::CombineArgs ca;

@@ -84,6 +84,11 @@ struct DecodeCfg {
   static constexpr int HT = QS == 1 ? 2 * NQ : NQ;  // score head slots per lane
   static_assert(RING_BYTES >= kWarps * 8 * D * 4, "merge buffer must fit in the ring");
   static_assert(WB_BYTES >= 8 * D * 4, "rotated queries must fit in the staging buffer");
+  // fused append: rows whose inputs one warp loads before quantizing them,
+  // and its shared scratch (one binary32 row and one row of codes)
+  static constexpr int APPEND_BATCH = 4;
+  static constexpr int APPEND_SCRATCH = 5 * D;
+  static_assert(WB_BYTES >= kWarps * APPEND_SCRATCH, "append scratch must fit in the staging buffer");
   static_assert(SLOT_BYTES % 16 == 0 && SLOT_K % 16 == 0 && SLOT_V % 16 == 0, "alignment");
   static_assert(GK >= 16 && GK % 16 == 0 && GV >= 16 && GV % 16 == 0,
                 "groups must cover whole 16-element steps");
@@ -208,7 +213,10 @@ __device__ __forceinline__ void store_out(void* out, int dtype, size_t i, float 
     reinterpret_cast<__half*>(out)[i] = __float2half_rn(v);
 }
 
-template <class C>
+// FUSED: the instance used by the fused append + decode call (the append
+// prologue is compiled only there, so the plain decode keeps its registers
+// and schedule).
+template <class C, bool FUSED>
 __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a) {
   constexpr int D = C::D, NGK = C::NGK, NGV = C::NGV, NQ = C::NQ, NP = C::NP, QS = C::QS;
   constexpr int HT = C::HT, KSTEPS = C::KSTEPS, GK = C::GK, GV = C::GV;
@@ -237,7 +245,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   // fused append: positions [len - n_new, len) are written first; a row
   // whose length is out of range appends nothing
   int app_pos = -1;
-  if (a.k_new != nullptr && len <= lim) {
+  if (FUSED && a.k_new != nullptr && len <= lim) {
     if (len < a.n_new) {
       if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0) flag_error(a.err, KVQ_DEVERR_BAD_POS);
     } else {
@@ -262,26 +270,6 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   const int t1 = min(t0 + a.split_tokens, len);
   const int n_tok = t1 - t0;
   const size_t slot = static_cast<size_t>(b) * a.kv_heads + hk;
-
-  // ---- fused append of the new positions in this split (every head-group
-  // CTA of the slot writes the same bytes), made visible to the bulk copies
-  // below before any is issued
-  if (app_pos >= 0) {
-    const int p0 = max(app_pos, t0), p1 = t1;
-    if (p0 < p1) {
-      auto row_of_pos = [&](int p) -> long long {
-        if (a.block_table == nullptr) return static_cast<long long>(slot) * a.capacity + p;
-        const int page = a.block_table[static_cast<size_t>(b) * a.pages_per_seq + (p >> a.page_shift)];
-        if (page < 0 || page >= a.num_pages) return -1;
-        return ((static_cast<long long>(page) * a.kv_heads + hk) << a.page_shift) +
-               (p & ((1 << a.page_shift) - 1));
-      };
-      append_rows<C>(a, b, hk, app_pos, p0, p1, smem + warp * 5 * D, row_of_pos);
-      fence_proxy_async_global();
-      __syncthreads();
-      fence_proxy_async_global();
-    }
-  }
 
   // ---- this warp's copy pipeline: positions [it*kStageTokens + 16*TPW*warp, +16*TPW)
   // of the split for it = 0 .. my_iters-1, kSlots copies in flight.
@@ -328,9 +316,44 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
                   reinterpret_cast<const uint8_t*>(a.v_params) + r * C::PROWV, pvbytes,
                   &wfull[sl]);
   };
+  // First stages.  With a fused append, the stages that end before the new
+  // positions go out first, so that their copies overlap the append.
+  int first_pending = min(C::kSlots, my_iters);
   if (lane == 0)
-    for (int it = 0; it < min(C::kSlots, my_iters); ++it)
+    for (int it = 0; it < min(C::kSlots, my_iters); ++it) {
+      if (FUSED && app_pos >= 0 && t0 + it * C::kStageTokens + my_first + 16 * C::TPW > app_pos) {
+        first_pending = it;
+        break;
+      }
       issue(it, it, a.block_table != nullptr ? page_of(it) : 0);
+    }
+  if constexpr (FUSED) {
+    // ---- fused append of the new positions in this split (every head-group
+    // CTA of the slot writes the same bytes), made visible to the bulk
+    // copies of the remaining stages before they are issued.  Scratch: the
+    // weight staging buffer, unused until the first tile.
+    if (app_pos >= 0) {
+      const int p0 = max(app_pos, t0), p1 = t1;
+      if (p0 < p1) {
+        auto row_of_pos = [&](int p) -> long long {
+          if (a.block_table == nullptr) return static_cast<long long>(slot) * a.capacity + p;
+          const int page =
+              a.block_table[static_cast<size_t>(b) * a.pages_per_seq + (p >> a.page_shift)];
+          if (page < 0 || page >= a.num_pages) return -1;
+          return ((static_cast<long long>(page) * a.kv_heads + hk) << a.page_shift) +
+                 (p & ((1 << a.page_shift) - 1));
+        };
+        append_rows<C>(a, b, hk, app_pos, p0, p1,
+                       reinterpret_cast<uint8_t*>(wbuf) + warp * C::APPEND_SCRATCH, row_of_pos);
+        fence_proxy_async_global();
+        __syncthreads();
+        fence_proxy_async_global();
+      }
+    }
+    if (lane == 0)
+      for (int it = first_pending; it < min(C::kSlots, my_iters); ++it)
+        issue(it, it, a.block_table != nullptr ? page_of(it) : 0);
+  }
   __syncwarp();
 
   // ------------------------------------------------------------ consumers
@@ -896,18 +919,20 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   }
 }
 
-template <class C>
+template <class C, bool FUSED>
 cudaError_t launch_decode(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
-  return launch_pdl(decode_kernel<C>, grid, dim3(C::kThreads), C::SMEM_BYTES, stream, a);
+  return launch_pdl(decode_kernel<C, FUSED>, grid, dim3(C::kThreads), C::SMEM_BYTES, stream, a);
 }
 
 template <class C>
 DecodeKernel make_decode_kernel() {
   DecodeKernel k;
-  k.fn = reinterpret_cast<const void*>(&decode_kernel<C>);
+  k.fn = reinterpret_cast<const void*>(&decode_kernel<C, false>);
+  k.fn_fused = reinterpret_cast<const void*>(&decode_kernel<C, true>);
   k.threads = C::kThreads;
   k.smem_bytes = C::SMEM_BYTES;
-  k.launch = &launch_decode<C>;
+  k.launch = &launch_decode<C, false>;
+  k.launch_fused = &launch_decode<C, true>;
   return k;
 }
 

@@ -90,10 +90,12 @@ struct DecodeArgs {
 //   0: 16-bit Q, <= 4 heads    1: fp32 Q, <= 4 heads
 //   2: 16-bit Q, 5..8 heads    3: fp32 Q, 5..8 heads
 struct DecodeKernel {
-  const void* fn;      // __global__ function
+  const void* fn;        // __global__ function
+  const void* fn_fused;  // the same with the fused append (k_new != NULL)
   int threads;
   int smem_bytes;
   cudaError_t (*launch)(const DecodeArgs&, dim3 grid, cudaStream_t stream);
+  cudaError_t (*launch_fused)(const DecodeArgs&, dim3 grid, cudaStream_t stream);
 };
 
 // Returns false if (D, bits, key groups, value groups, variant) has no instance.
