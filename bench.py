@@ -86,7 +86,8 @@ KERNEL_SOURCES = {
     "quantize": ["kv_cache_mixed_kvq_b200/csrc/quantize.cuh", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
     "quantize_rot": ["kv_cache_mixed_kvq_b200/csrc/quantize.cuh",
                      "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
-    "decode": ["kv_cache_mixed_kvq_b200/csrc/decode.cuh", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
+    "decode": ["kv_cache_mixed_kvq_b200/csrc/decode.cuh", "kv_cache_mixed_kvq_b200/csrc/append_rows.cuh",
+               "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
     "combine": ["kv_cache_mixed_kvq_b200/csrc/combine.cu", "kv_cache_mixed_kvq_b200/csrc/common.cuh"],
 }
 
