@@ -86,7 +86,7 @@ __device__ __forceinline__ void quantize_row_warp(const float (&x)[D / 32], uint
 // per-position arrays, or -1 when the block table names no page (the row is
 // skipped and flagged).
 template <class C, class RowOf>
-__device__ __noinline__ void append_rows(const DecodeArgs& a, int b, int hk, int pos, int p0,
+__device__ __forceinline__ void append_rows(const DecodeArgs& a, int b, int hk, int pos, int p0,
                                          int p1, uint8_t* stage, RowOf row_of) {
   constexpr int D = C::D, PER = D / 32, NB = C::APPEND_BATCH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
