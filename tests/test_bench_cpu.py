@@ -87,3 +87,13 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert res["impl"] == "reference" and res["value"] > 0 and res["unit"] == "GB/s"
     assert res["cpu_baseline"]["kind"] == "oracle"
     assert res["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_cpu_baseline_uses_every_core_and_splits_the_phases():
+    import bench
+    w = bench.workloads.WORKLOADS["tiny"]
+    res = bench.cpu_baseline(w, w.bits[0], 0.5)
+    assert res["kind"] == "oracle" and res["value"] > 0
+    assert res["cores"] == bench.host_cores()
+    single = res["single_thread"]
+    assert single["cores"] == 1 and single["quantize_gbs"] > 0 and single["decode_gbs"] > 0
