@@ -542,11 +542,17 @@ def _oracle_row(_):
     return oracle_run(w, bits, inputs)
 
 
+MAX_ORACLE_PROCS = 16  # each worker process imports torch: bounded host memory and start-up
+
+
 def host_cores() -> int:
+    """Host cores the oracle pool uses: the cores this process may run on, at
+    most MAX_ORACLE_PROCS."""
     try:
-        return len(os.sched_getaffinity(0))
+        n = len(os.sched_getaffinity(0))
     except AttributeError:
-        return os.cpu_count() or 1
+        n = os.cpu_count() or 1
+    return max(1, min(n, MAX_ORACLE_PROCS))
 
 
 class OraclePool:
