@@ -90,7 +90,8 @@
  * a length above `max_seq_len` or `capacity`, a bounded wait that ran out)
  * set bits in a per-device error word that kvq_device_error_flags() reads and
  * clears; the offending rows are skipped or clamped, never written out of
- * bounds.  Layouts of K, V, Q and out are row-major with head_dim innermost.
+ * bounds.  A paged cache's block-table entries are device data too: an entry
+ * outside the pool is flagged and never followed.  Layouts of K, V, Q and out are row-major with head_dim innermost.
  */
 #ifndef KVQ_H_
 #define KVQ_H_

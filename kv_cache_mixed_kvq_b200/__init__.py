@@ -12,6 +12,11 @@ Typical use::
                              bits_k=4, bits_v=2, group=64, device="cuda")
     kvq_quantize_append(cache, k, v, pos)            # k, v: [B][Hkv][n][D]
     out = kvq_decode_attention(cache, q, seq_lens, max_seq_len)   # q: [B][Hq][D]
+    # or both in one launch, the new rows at seq_lens - n .. seq_lens - 1:
+    out = kvq_append_decode_attention(cache, k, v, q, seq_lens, max_seq_len)
+
+A paged cache (block tables) is allocated with ``page_size``, ``num_pages``
+and an int32 ``block_table`` [batch][capacity / page_size].
 """
 from __future__ import annotations
 

@@ -30,7 +30,12 @@
 //    partial results per split are merged by a separate log-sum-exp combine,
 //    except when a row has a single split: its CTA then writes the output;
 //  * with rotated keys (KVQ_FLAG_ROTATE_KEYS) the prologue turns the query
-//    into H q / D in shared memory.
+//    into H q / D in shared memory;
+//  * paged layout (KVQ_FLAG_PAGED): a stage's 32 positions lie in one page;
+//    lane 0 looks the page up in the block table one stage ahead;
+//  * the FUSED instances (kvq_append_decode_attention) first quantize and
+//    write the step's new positions that fall in the CTA's split (see
+//    append_rows.cuh), then stream as above.
 #pragma once
 
 #include <type_traits>
