@@ -228,3 +228,48 @@ def test_zero_new_tokens_is_plain_decode(ora):
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     assert all(torch.equal(x, y) for x, y in zip(before, (cache.k_codes, cache.v_codes)))
+
+
+@pytest.mark.parametrize("n_new,lens", [(100, (100, 230, 164)), (64, (64, 128, 65))])
+def test_fused_append_spans_several_splits(ora, n_new, lens):
+    # more new tokens than a split holds (64): several CTAs of one slot each
+    # write their own part; rows whose length equals n_new append at 0
+    cache, hc, out, ref, flags, _ = _fused_case(ora, n_new=n_new, split=64, lens=lens, gq=16)
+    assert flags == 0 and kvq.kvq_device_error_flags() == 0
+    assert_same_cache(cache, hc)
+    compare_attention(out, ref, TOL)
+
+
+def test_fused_everything_at_once(ora):
+    # rotated keys, coarser value groups, paged pool, f16 inputs, fp32 queries
+    cache, hc, out, ref, flags, _ = _fused_case(ora, G=32, gv=128, n_new=21, split=64,
+                                                rotate=True, page_size=64, lens=(150, 21, 256),
+                                                dtype=torch.float16, q_dtype=torch.float32)
+    assert flags == 0 and kvq.kvq_device_error_flags() == 0
+    assert_same_cache(cache, hc)
+    compare_attention(out, ref, TOL)
+
+
+def test_fused_bad_page_is_flagged_not_followed(ora):
+    B, Hkv, D, cap, P, n_new = 2, 2, 128, 256, 64, 8
+    table = np.array([[0, 1, -1, 6], [2, 3, 4, 5]], np.int32)   # row 0: entries 2, 3 bad
+    cache = kvq.KVCache.allocate(B, Hkv, D, cap, 4, 2, 64, page_size=P, num_pages=6,
+                                 block_table=torch.from_numpy(table))
+    hc = ora.PagedHostCache(B, Hkv, D, cap, 4, 2, 64, P, 6, table)
+    _prefill(ora, cache, hc, [120, 120], D, seed=9, dtype=torch.bfloat16)
+    k, v = _inputs(B, Hkv, n_new, D, seed=10)
+    q = torch.randn(B, 2 * Hkv, D, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    lens = [133, 128]   # row 0's new positions 125..132 reach entry 2
+    kb, dt = workloads.as_bits(k)
+    vb, _ = workloads.as_bits(v)
+    qb, qdt = workloads.as_bits(q)
+    ref, flags = ora.append_decode_attention(hc, kb, vb, qb, 2 * Hkv, lens, dtype=dt,
+                                             q_dtype=qdt, max_len=cap)
+    assert flags == kvq.KVQ_DEVERR_BAD_PAGE
+    out = kvq.kvq_append_decode_attention(cache, k.cuda(), v.cuda(), q.cuda(),
+                                          torch.tensor(lens, dtype=torch.int32, device="cuda"),
+                                          cap, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert kvq.kvq_device_error_flags() == kvq.KVQ_DEVERR_BAD_PAGE
+    assert_same_cache(cache, hc)          # the valid pages hold the same bytes
+    compare_attention(out[1:], ref[1:], TOL)   # row 0's output is unspecified
