@@ -9,8 +9,8 @@ layer (batch 8, 32 query / 8 KV heads, head_dim 128, 4096 tokens per
 sequence, bf16, K4V2, group 64), quantizing the full cache then one decode
 step.  Other workloads (`--workload`) append their new tokens and decode.
 
-Timing: inputs and caches rotate over enough sets that no step finds its data
-in L2; each step is replayed from a CUDA graph; the timed region is bracketed
+Timing: inputs and caches rotate over enough sets (at least --rotate) that
+the data touched between two uses of a set exceeds twice the L2; each step is replayed from a CUDA graph; the timed region is bracketed
 by a barrier and a device synchronize, timed with CUDA events on the launch
 stream, max over ranks.  Prints one JSON line (rank 0).
 
@@ -269,11 +269,25 @@ def _slot_view(cache, b):
                        rotate_keys=cache.rotate_keys, group_v=cache.group_v)
 
 
+L2_BYTES = 126 * 2**20
+MAX_SETS = 16
+
+
+def sets_needed(step_bytes: float, at_least: int) -> int:
+    """Rotating input/cache sets so that the other sets' data, touched between
+    two uses of one set, exceed twice the L2 (at most MAX_SETS; a step whose
+    data is far below the L2 then still finds some of it there)."""
+    need = 1 + -(-2 * L2_BYTES // max(int(step_bytes), 1))
+    return max(at_least, min(need, MAX_SETS))
+
+
 def run_ours(args, rank, world, device):
     w = workloads.WORKLOADS[args.workload]
     bits = tuple(int(x) for x in args.bits.split(",")) if args.bits else w.bits[-1] \
         if w.name == "long" else w.bits[0]
-    rotate = args.rotate
+    n_new0, _, read0 = step_shape(w, bits)
+    nb0 = algorithmic_bytes(w, bits, n_new0, read0, args.group_v)
+    rotate = sets_needed(nb0["quantize"] * (1 if n_new0 else 0) + nb0["decode"], args.rotate)
     arm = Arm(w, bits, rotate, device, rotate_keys=args.rotate_keys, group_v=args.group_v,
               page_size=args.page_size, fused=args.fused)
     stream = torch.cuda.current_stream()
@@ -369,8 +383,8 @@ def run_ours(args, rank, world, device):
                      f"append {arm.n_new} inside the decode + combine" if arm.fused else
                      f"append {arm.n_new} + decode + combine"),
             "split_tokens": arm.split_tokens,
-            "l2": f"{rotate} rotating input/cache sets (each step's data last touched "
-                  f"{rotate - 1} steps earlier), graph replay",
+            "l2": f"{rotate} rotating input/cache sets of {step_bytes / 1e6:.1f} MB (each "
+                  f"step's data last touched {rotate - 1} steps earlier), graph replay",
             "parallelism": f"replicas{world}" if world > 1 else "single",
         },
         "kv_tokens_per_s": round(world * nbytes["tokens"] / (ms_step / 1e3), 1),

@@ -97,3 +97,14 @@ def test_cpu_baseline_uses_every_core_and_splits_the_phases():
     assert res["cores"] == bench.host_cores()
     single = res["single_thread"]
     assert single["cores"] == 1 and single["quantize_gbs"] > 0 and single["decode_gbs"] > 0
+
+
+def test_rotation_exceeds_twice_the_l2():
+    import bench
+    for step_bytes in (1e3, 29.4e6, 118e6, 193e6, 248e6, 1e9):
+        n = bench.sets_needed(step_bytes, 3)
+        assert 3 <= n <= bench.MAX_SETS
+        if n < bench.MAX_SETS:
+            assert (n - 1) * step_bytes >= 2 * bench.L2_BYTES
+    assert bench.sets_needed(193e6, 3) == 3      # the default workload keeps three sets
+    assert bench.sets_needed(29.4e6, 3) == 10
