@@ -1,21 +1,31 @@
 #!/usr/bin/env python
 """Benchmark of the mixed-precision KV-cache hot path on B200.
 
-One step = one pass of the whole path over one batch of synthetic input:
-quantize-append (group-wise min-max, keys at b_k and values at b_v bits,
-bit-packed) followed by split-K decode attention over the packed cache and
-the log-sum-exp combine.  Default workload: the Llama-3-8B-shaped decode
-layer (batch 8, 32 query / 8 KV heads, head_dim 128, 4096 tokens per
-sequence, bf16, K4V2, group 64), quantizing the full cache then one decode
-step.  Other workloads (`--workload`) append their new tokens and decode.
+The metric is decode attention over the packed cache: the split-K decode
+kernel plus the log-sum-exp combine, in algorithmic HBM GB/s (the packed
+cache bytes the step must read, plus the query read and the output write)
+and KV tokens per second.  Default workload: the ragged batch (64 sequences,
+lengths uniform in [512, 8192] from seed 0, 32 query / 8 KV heads,
+head_dim 128, K4V2, group 64), the largest configuration, whose step is one
+decode step over a resident cache.  Other workloads (`--workload`) time
+their own step: the Llama-3-8B-shaped layer quantizes its full cache and then
+decodes; the long-context and Qwen/Mistral-shaped layers append their new
+tokens and decode.
 
-Timing: inputs and caches rotate over enough sets (at least --rotate) that
-the data touched between two uses of a set exceeds twice the L2; each step is replayed from a CUDA graph; the timed region is bracketed
-by a barrier and a device synchronize, timed with CUDA events on the launch
+After the timed region the same JSON line records every configuration
+(all workloads and bit pairs) under "configs": the device time of each of
+its kernels (median of at least 50 isolated graph replays) with its
+algorithmic bytes, GB/s and fraction of the measured HBM copy bandwidth.
+
+Timing: inputs and caches rotate over enough sets that the data touched
+between two uses of a set exceeds twice the L2 (the device's own L2 size);
+each step is replayed from a CUDA graph; the timed region is bracketed by a
+barrier and a device synchronize, timed with CUDA events on the launch
 stream, max over ranks.  Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME] [--bits K,V] [--group-v G] [--rotate-keys]
+                  [--page-size P] [--fused] [--no-configs]
 """
 from __future__ import annotations
 
@@ -39,6 +49,11 @@ from kv_cache_mixed_kvq_b200 import workloads  # noqa: E402
 
 METRIC = "quantized-KV decode attention HBM GB/s (% of B200 peak) and KV-tokens/s, K4V2"
 FALLBACK_HBM_GBS = 6650.0
+DEFAULT_WORKLOAD = "ragged"
+# every (workload, bits) configuration, recorded in the "configs" key
+CONFIG_SWEEP = (("tiny", (4, 2)), ("llama3_8b", (4, 2)), ("long", (8, 4)), ("long", (4, 2)),
+                ("ragged", (4, 2)), ("qwen_mistral", (4, 2)), ("qwen_mistral", (2, 4)))
+KERNEL_REPS = 60  # isolated graph replays per kernel time (median)
 
 
 # --------------------------------------------------------------- workload
@@ -269,27 +284,105 @@ def _slot_view(cache, b):
                        rotate_keys=cache.rotate_keys, group_v=cache.group_v)
 
 
-L2_BYTES = 126 * 2**20
 MAX_SETS = 16
 
 
-def sets_needed(step_bytes: float, at_least: int) -> int:
+def l2_bytes(device) -> int:
+    """L2 size of the device, from its properties."""
+    return int(torch.cuda.get_device_properties(device).L2_cache_size)
+
+
+def sets_needed(step_bytes: float, at_least: int, l2: int) -> int:
     """Rotating input/cache sets so that the other sets' data, touched between
     two uses of one set, exceed twice the L2 (at most MAX_SETS; a step whose
     data is far below the L2 then still finds some of it there)."""
-    need = 1 + -(-2 * L2_BYTES // max(int(step_bytes), 1))
+    need = 1 + -(-2 * l2 // max(int(step_bytes), 1))
     return max(at_least, min(need, MAX_SETS))
+
+
+def default_bits(w):
+    return w.bits[-1] if w.name == "long" else w.bits[0]
+
+
+def make_arm(w, bits, device, at_least: int, **kw):
+    """An Arm whose rotation exceeds twice the L2, and its algorithmic bytes."""
+    n_new0, _, read0 = step_shape(w, bits)
+    nb0 = algorithmic_bytes(w, bits, n_new0, read0, kw.get("group_v", 0))
+    rotate = sets_needed(nb0["quantize"] * (1 if n_new0 else 0) + nb0["decode"], at_least,
+                         l2_bytes(device))
+    return Arm(w, bits, rotate, device, **kw), rotate
+
+
+def roofline_entry(name, ms, kbytes, hbm_peak, peak_kind, traffic, reps):
+    ach = kbytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(ach / hbm_peak, 4), "traffic": traffic, "ms": round(ms, 5),
+            "algorithmic_bytes": kbytes, "timing": f"median of {reps} isolated graph replays",
+            "peak_source": f"{peak_kind} hbm_gbs (copy)"}
+
+
+def kernel_rooflines(arm, w, kern, nbytes, reps, rotate_keys=False):
+    """Roofline objects of the step's kernels from their median device times."""
+    hbm_peak, peak_kind = peaks()
+    roof = {}
+    if "quantize" in kern:
+        roof["quantize"] = roofline_entry(
+            "quantize", kern["quantize"], nbytes["quantize"], hbm_peak, peak_kind,
+            measured_traffic(["quantize_rot" if rotate_keys else "quantize"], w.name), reps)
+    # the fused call also moves the append's bytes
+    kbytes = nbytes["decode"] + (nbytes["quantize"] if arm.fused else 0)
+    roof["decode_attention"] = roofline_entry(
+        "decode_attention", kern["decode_attention"], kbytes, hbm_peak, peak_kind,
+        None if arm.fused else measured_traffic(
+            ["decode"] if arm.num_splits == 1 else ["decode", "combine"], w.name), reps)
+    roof["decode_attention"]["kernels"] = ("decode (with the append fused)" if arm.fused else
+                                           "decode" if arm.num_splits == 1 else
+                                           "decode + combine")
+    return roof
+
+
+def measure_config(name, bits, device, reps):
+    """Per-kernel device times and rooflines of one configuration's step."""
+    w = workloads.WORKLOADS[name]
+    arm, rotate = make_arm(w, bits, device, 3)
+    for i in range(3):
+        arm.step(i % rotate)
+    torch.cuda.synchronize()
+    kern = per_kernel_times(arm, rotate, reps)
+    flags = arm.kvq.kvq_device_error_flags()
+    nbytes = algorithmic_bytes(w, bits, arm.n_new, arm.read)
+    roof = kernel_rooflines(arm, w, kern, nbytes, reps)
+    dec = roof["decode_attention"]
+    entry = {
+        "workload": name, "bits": f"K{bits[0]}V{bits[1]}",
+        "step": step_name(w, arm),
+        "split_tokens": arm.split_tokens, "num_splits": arm.num_splits,
+        "rotating_sets": rotate,
+        "kv_tokens": nbytes["tokens"],
+        "decode_kv_tokens_per_s": round(nbytes["tokens"] / (dec["ms"] / 1e3), 1),
+        "kernels": roof,
+        "device_error_flags": flags,
+    }
+    del arm
+    torch.cuda.empty_cache()
+    return entry
+
+
+def step_name(w, arm):
+    if w.name == "llama3_8b":
+        return "quantize full cache + decode + combine"
+    if arm.fused:
+        return f"append {arm.n_new} inside the decode + combine"
+    if arm.n_new:
+        return f"append {arm.n_new} + decode + combine"
+    return "decode + combine (one decode step over the resident cache)"
 
 
 def run_ours(args, rank, world, device):
     w = workloads.WORKLOADS[args.workload]
-    bits = tuple(int(x) for x in args.bits.split(",")) if args.bits else w.bits[-1] \
-        if w.name == "long" else w.bits[0]
-    n_new0, _, read0 = step_shape(w, bits)
-    nb0 = algorithmic_bytes(w, bits, n_new0, read0, args.group_v)
-    rotate = sets_needed(nb0["quantize"] * (1 if n_new0 else 0) + nb0["decode"], args.rotate)
-    arm = Arm(w, bits, rotate, device, rotate_keys=args.rotate_keys, group_v=args.group_v,
-              page_size=args.page_size, fused=args.fused)
+    bits = tuple(int(x) for x in args.bits.split(",")) if args.bits else default_bits(w)
+    arm, rotate = make_arm(w, bits, device, args.rotate, rotate_keys=args.rotate_keys,
+                           group_v=args.group_v, page_size=args.page_size, fused=args.fused)
     stream = torch.cuda.current_stream()
 
     # warm-up (also loads every kernel and the error-word address)
@@ -317,9 +410,7 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device() if not os.environ.get("CUDA_VISIBLE_DEVICES")
-                      else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[
-                          torch.cuda.current_device()])) as clocks:
+    with ClockSampler(physical_index()) as clocks:
         t0.record(stream)
         for i in range(args.steps):
             graphs[i % rotate].replay()
@@ -335,33 +426,36 @@ def run_ours(args, rank, world, device):
     step_bytes = nbytes["quantize"] * (1 if arm.n_new else 0) + nbytes["decode"]
 
     # ---------------- per-kernel durations (events inside a graph, GPU kept busy)
-    kern = per_kernel_times(arm, rotate, stream, reps=max(10, min(args.steps, 40)))
-    hbm_peak, peak_kind = peaks()
-    roof = {}
-    for name, key in (("quantize", "quantize"), ("decode_attention", "decode")):
-        if name not in kern:
-            continue
-        t_s = kern[name] / 1e3
-        # the fused call also moves the append's bytes
-        kbytes = nbytes[key] + (nbytes["quantize"] if arm.fused and key == "decode" else 0)
-        ach = kbytes / t_s / 1e9
-        roof[name] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak,
-                      "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
-                      "traffic": measured_traffic(
-                          (["quantize_rot"] if args.rotate_keys else ["quantize"])
-                          if key == "quantize" else
-                          (["decode"] if arm.num_splits == 1 else ["decode", "combine"]), w.name),
-                      "ms": round(kern[name], 5), "algorithmic_bytes": kbytes,
-                      "peak_source": f"{peak_kind} hbm_gbs (copy)"}
-    dominant = "quantize" if "quantize" in roof and kern["quantize"] >= kern.get(
-        "decode_attention", 0) else "decode_attention"
+    with ClockSampler(physical_index()) as kclocks:
+        kern = per_kernel_times(arm, rotate, KERNEL_REPS)
+    roof = kernel_rooflines(arm, w, kern, nbytes, KERNEL_REPS, args.rotate_keys)
 
     # ---------------- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(arm, args, step_bytes, world, device)
+    graphs.clear()  # release the graphs before any process-group teardown
 
     probe = read_probe_gbs(device)
+    cfg = {
+        "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+        "head_dim": w.head_dim, "context": w.context, "input_dtype": w.dtype,
+        "bits_k": bits[0], "bits_v": bits[1], "group": w.group,
+        "rotate_keys": bool(args.rotate_keys),
+        "group_v": args.group_v or w.group,
+        "page_size": args.page_size,
+        "fused_append": arm.fused,
+        "step": step_name(w, arm),
+        "kv_tokens_per_step": nbytes["tokens"],
+        "split_tokens": arm.split_tokens,
+        "l2": f"{rotate} rotating input/cache sets of {step_bytes / 1e6:.1f} MB (each "
+              f"step's data last touched {rotate - 1} steps earlier; L2 "
+              f"{l2_bytes(device) / 2**20:.0f} MiB), graph replay",
+        "parallelism": f"replicas{world}" if world > 1 else "single",
+    }
+    if w.ragged:
+        cfg["seq_lens"] = f"uniform in [{w.ragged[0]}, {w.ragged[1]}] from seed 0, " \
+                          f"sum {nbytes['tokens']}, max {arm.max_len}"
     result = {
         "metric": METRIC,
         "value": round(world * step_bytes / (ms_step / 1e3) / 1e9, 2),
@@ -369,26 +463,12 @@ def run_ours(args, rank, world, device):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32",
+        "dtype": "f16-mma/f32",
         "data": "synthetic",
-        "config": {
-            "workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
-            "head_dim": w.head_dim, "context": w.context, "input_dtype": w.dtype,
-            "bits_k": bits[0], "bits_v": bits[1], "group": w.group,
-            "rotate_keys": bool(args.rotate_keys),
-            "group_v": args.group_v or w.group,
-            "page_size": args.page_size,
-            "fused_append": arm.fused,
-            "step": ("quantize full cache + decode + combine" if w.name == "llama3_8b" else
-                     f"append {arm.n_new} inside the decode + combine" if arm.fused else
-                     f"append {arm.n_new} + decode + combine"),
-            "split_tokens": arm.split_tokens,
-            "l2": f"{rotate} rotating input/cache sets of {step_bytes / 1e6:.1f} MB (each "
-                  f"step's data last touched {rotate - 1} steps earlier), graph replay",
-            "parallelism": f"replicas{world}" if world > 1 else "single",
-        },
+        "config": cfg,
         "kv_tokens_per_s": round(world * nbytes["tokens"] / (ms_step / 1e3), 1),
-        "roofline": dict(roof[dominant], kernel=dominant),
+        # the metric's own kernel(s): decode attention
+        "roofline": dict(roof["decode_attention"], kernel="decode_attention"),
         "read_probe": {"value": probe, "unit": "GB/s",
                        "what": "torch sum over 1 GiB fp32, best of 10 (context, not the peak)"},
         "roofline_by_kernel": roof,
@@ -396,15 +476,30 @@ def run_ours(args, rank, world, device):
         "device_error_flags": flags,
         "e2e": e2e,
         "clocks": clocks.summary(),
-        "arith": "binary32 quantizer; exact integer codes x binary16 operands on tensor "
-                 "cores with binary32 accumulation; binary32 softmax",
+        "clocks_kernel_timing": kclocks.summary(),
+        "arith": "binary32 quantizer; exact integer codes as binary16 tensor-core operands "
+                 "against binary16 high/low splits of the query and of the output weights, "
+                 "binary32 accumulation; binary32 softmax",
     }
+    del arm
+    torch.cuda.empty_cache()
+    if not args.no_configs:
+        with ClockSampler(physical_index()) as cclocks:
+            result["configs"] = [measure_config(n, b, device, KERNEL_REPS)
+                                 for n, b in CONFIG_SWEEP]
+        result["clocks_configs"] = cclocks.summary()
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, bits, args.cpu_seconds)
-    if world > 1:
-        for g in graphs:
-            del g
     return result
+
+
+def physical_index():
+    """nvidia-smi index of the current device."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    cur = torch.cuda.current_device()
+    if not vis:
+        return cur
+    return int(vis.split(",")[cur])
 
 
 def read_probe_gbs(device, nbytes=1 << 30, reps=10):
@@ -426,10 +521,11 @@ def read_probe_gbs(device, nbytes=1 << 30, reps=10):
     return round(nbytes / (best / 1e3) / 1e9, 1)
 
 
-def per_kernel_times(arm, rotate, stream, reps):
-    """Average device time of the quantize launch and of the decode-attention
-    call (decode + combine), from events captured inside per-set graphs; a
-    sleep kernel keeps the GPU busy so that launch gaps are not timed."""
+def per_kernel_times(arm, rotate, reps):
+    """Median device time of the quantize launch and of the decode-attention
+    call (decode + combine) over `reps` replays, from events captured inside
+    per-set graphs; a sleep kernel keeps the GPU busy before each replay so
+    that launch gaps are not timed."""
     evs, graphs = [], []
     for r in range(rotate):
         e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
@@ -451,35 +547,40 @@ def per_kernel_times(arm, rotate, stream, reps):
         e = evs[r]
         q.append(e[0].elapsed_time(e[1]))
         d.append(e[1].elapsed_time(e[2]))
-    out = {"decode_attention": statistics.mean(d)}
+    out = {"decode_attention": statistics.median(d)}
     if arm.n_new and not arm.fused:
-        out["quantize"] = statistics.mean(q)
+        out["quantize"] = statistics.median(q)
     return out
 
 
 def run_e2e(arm, args, step_bytes, world, device):
     """Same step through the public API with pinned host buffers: H2D of the
-    step's inputs, quantize + decode, D2H of the output, every step."""
+    step's inputs (query, lengths and any new K/V rows), the step's calls,
+    D2H of the output, every step.  The cache is the step's resident state."""
     s0 = arm.sets[0]
     hk = s0["k"].cpu().pin_memory()
     hv = s0["v"].cpu().pin_memory()
     hq = s0["q"].cpu().pin_memory()
+    hlens = arm.lens.cpu().pin_memory()
     hout = torch.empty_like(s0["out"], device="cpu").pin_memory()
     k_dev, v_dev, q_dev = torch.empty_like(s0["k"]), torch.empty_like(s0["v"]), torch.empty_like(s0["q"])
+    lens_dev = torch.empty_like(arm.lens)
     cache = s0["cache"]
     stream = torch.cuda.current_stream()
 
     def one():
-        k_dev.copy_(hk, non_blocking=True)
-        v_dev.copy_(hv, non_blocking=True)
+        if arm.n_new:
+            k_dev.copy_(hk, non_blocking=True)
+            v_dev.copy_(hv, non_blocking=True)
         q_dev.copy_(hq, non_blocking=True)
+        lens_dev.copy_(hlens, non_blocking=True)
         if arm.fused:
-            arm.kvq.kvq_append_decode_attention(cache, k_dev, v_dev, q_dev, arm.lens,
+            arm.kvq.kvq_append_decode_attention(cache, k_dev, v_dev, q_dev, lens_dev,
                                                 arm.max_len, out=s0["out"], workspace=arm.ws)
         else:
             if arm.n_new:
                 arm.kvq.kvq_quantize_append(cache, k_dev, v_dev, arm.pos_t)
-            arm.kvq.kvq_decode_attention(cache, q_dev, arm.lens, arm.max_len, out=s0["out"],
+            arm.kvq.kvq_decode_attention(cache, q_dev, lens_dev, arm.max_len, out=s0["out"],
                                          workspace=arm.ws)
         hout.copy_(s0["out"], non_blocking=True)
 
@@ -496,64 +597,92 @@ def run_e2e(arm, args, step_bytes, world, device):
     b.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b) / steps, world, device)
-    h2d = (hk.numel() * hk.element_size() + hv.numel() * hv.element_size() +
-           hq.numel() * hq.element_size()) if arm.n_new else hq.numel() * hq.element_size()
+    h2d = hq.numel() * hq.element_size() + hlens.numel() * hlens.element_size()
+    if arm.n_new:
+        h2d += hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
     return {"value": round(world * step_bytes / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 4), "steps": steps,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+            "what": "the same step through the public API: pinned host query and lengths "
+                    "(and new K/V rows when the step appends) copied in, the output copied "
+                    "out, every step; the cache stays resident on the device"}
 
 
 # ---------------------------------------------------------- oracle (CPU)
-def oracle_inputs(w, bits, batch_rows, seed=0):
-    """Inputs of one oracle pass over `batch_rows` batch rows (bit patterns)."""
-    n_new, pos, read = step_shape(w, bits)
-    ks, vs = workloads.make_kv(w, max(read[:batch_rows]), seed=seed, batch=batch_rows)
-    q = workloads.make_q(w, seed=seed, batch=batch_rows)
-    kb, dt = workloads.as_bits(ks)
-    vb, _ = workloads.as_bits(vs)
-    qb, _ = workloads.as_bits(q)
-    return kb, vb, qb, dt, read[:batch_rows]
+def step_quantizes(w) -> bool:
+    """Whether the workload's step runs the quantizer (else it only decodes)."""
+    return w.name == "llama3_8b" or w.append > 0
 
 
-def oracle_run(w, bits, inputs):
-    """One oracle pass (quantize, then decode) over prepared inputs.  Returns
-    (quantize seconds, decode seconds, quantize bytes, decode bytes, KV tokens
-    read): algorithmic bytes of that sample."""
-    import oracle
-    kb, vb, qb, dt, read = inputs
-    rows = len(read)
-    cap = (max(read) + 15) // 16 * 16
-    hc = oracle.HostCache(rows, w.kv_heads, w.head_dim, cap, bits[0], bits[1], w.group)
-    t0 = time.perf_counter()
-    hc.quantize_append(kb, vb, [0] * rows, dtype=dt)
-    t1 = time.perf_counter()
-    hc.decode_attention(qb, w.q_heads, read, q_dtype=dt)
-    t2 = time.perf_counter()
-    nb = algorithmic_bytes(w, bits, max(read), read)
-    scale = rows / w.batch
-    # the oracle always quantizes the whole sample (a prefill), like the default step
-    return t1 - t0, t2 - t1, nb["quantize"] * scale, nb["decode"] * scale, sum(read)
+def row_bytes(w, bits, length):
+    """Algorithmic bytes of one batch row of `length` tokens: (quantize of its
+    whole context, decode of all its query heads)."""
+    bk, bv = bits
+    D, G = w.head_dim, w.group
+    el = 4 if w.dtype == "f32" else 2
+    per_tok = D * (bk + bv) // 8 + 2 * (D // G) * 4
+    quant = w.kv_heads * length * (2 * D * el + per_tok) + 4
+    decode = length * w.kv_heads * per_tok + 2 * w.q_heads * D * el + 4
+    return quant, decode
 
 
-def oracle_step(w, bits, batch_rows, seed=0):
-    return oracle_run(w, bits, oracle_inputs(w, bits, batch_rows, seed))
+class OracleRow:
+    """One batch row of the workload prepared for the oracle: its inputs
+    (bit patterns) and, for decode-only steps, its cache already quantized
+    (untimed: the step reads a resident cache)."""
+
+    def __init__(self, w, bits, row, seed):
+        import oracle
+        self.w, self.bits = w, bits
+        self.length = int(workloads.seq_lens(w)[row % w.batch])
+        ks, vs = workloads.make_kv(w, self.length, seed=seed, batch=1)
+        q = workloads.make_q(w, seed=seed, batch=1)
+        self.kb, self.dt = workloads.as_bits(ks)
+        self.vb, _ = workloads.as_bits(vs)
+        self.qb, _ = workloads.as_bits(q)
+        self.cap = (self.length + 15) // 16 * 16
+        self.hc = None
+        if not step_quantizes(w):
+            self.hc = self._quantized(oracle)
+
+    def _quantized(self, oracle):
+        w, bits = self.w, self.bits
+        hc = oracle.HostCache(1, w.kv_heads, w.head_dim, self.cap, bits[0], bits[1], w.group)
+        hc.quantize_append(self.kb, self.vb, [0], dtype=self.dt)
+        return hc
+
+    def run(self):
+        """One timed oracle pass: (quantize s, decode s, quantize bytes, decode
+        bytes, KV tokens).  Decode-only steps time the decode alone."""
+        import oracle
+        tq, bq = 0.0, 0
+        hc = self.hc
+        if hc is None:
+            t0 = time.perf_counter()
+            hc = self._quantized(oracle)
+            tq = time.perf_counter() - t0
+            bq = row_bytes(self.w, self.bits, self.length)[0]
+        t1 = time.perf_counter()
+        hc.decode_attention(self.qb, self.w.q_heads, [self.length], q_dtype=self.dt)
+        td = time.perf_counter() - t1
+        return tq, td, bq, row_bytes(self.w, self.bits, self.length)[1], self.length
 
 
-_POOL_TASK = None
+_POOL_ROW = None
 
 
 def _oracle_init(name, bits):
-    """Pool worker set-up: one batch row's inputs, drawn from the worker's pid
-    (so workers differ), generated before any timed task."""
-    global _POOL_TASK
+    """Pool worker set-up: one batch row (index and seed from the worker's
+    pid, so that workers cover the workload's length mix), prepared before
+    any timed task."""
+    global _POOL_ROW
     w = workloads.WORKLOADS[name]
-    _POOL_TASK = (w, bits, oracle_inputs(w, bits, 1, seed=os.getpid() % 1000))
+    _POOL_ROW = OracleRow(w, bits, os.getpid(), seed=os.getpid() % 1000)
 
 
 def _oracle_row(_):
-    """Pool worker: one single-row oracle pass on the worker's inputs."""
-    w, bits, inputs = _POOL_TASK
-    return oracle_run(w, bits, inputs)
+    """Pool worker: one single-row oracle pass on the worker's row."""
+    return _POOL_ROW.run()
 
 
 MAX_ORACLE_PROCS = 16  # each worker process imports torch: bounded host memory and start-up
@@ -570,7 +699,7 @@ def host_cores() -> int:
 
 
 class OraclePool:
-    """Single-row oracle steps on every host core: one process per core,
+    """Single-row oracle passes on every host core: one process per core,
     started with `spawn` (never forked from a process that has used CUDA)."""
 
     def __init__(self, procs: int, w, bits):
@@ -591,6 +720,11 @@ class OraclePool:
         self.pool.join()
 
 
+def what_sample(w):
+    return ("quantize its full context + decode all its query heads" if step_quantizes(w) else
+            "decode all its query heads over its resident quantized cache")
+
+
 def cpu_baseline(w, bits, budget_s):
     """The oracle on the host's cores: single-threaded (quantize and decode
     timed separately) for about budget_s / 2, then one row per process on
@@ -600,17 +734,19 @@ def cpu_baseline(w, bits, budget_s):
     sq = sd = bq = bd = 0.0
     toks, runs = 0, 0
     while sq + sd < budget_s / 2 or runs == 0:
-        a, b, c, d, t = oracle_step(w, bits, 1, seed=runs)
+        a, b, c, d, t = OracleRow(w, bits, runs, seed=runs).run()
         sq, sd, bq, bd, toks, runs = sq + a, sd + b, bq + c, bd + d, toks + t, runs + 1
     single = {"value": round((bq + bd) / (sq + sd) / 1e9, 4), "unit": "GB/s", "cores": 1,
-              "quantize_gbs": round(bq / sq / 1e9, 4), "decode_gbs": round(bd / sd / 1e9, 4),
+              "decode_gbs": round(bd / sd / 1e9, 4),
               "kv_tokens_per_s": round(toks / (sq + sd), 1),
               "sample": f"{runs} x one batch row of {w.name}, {sq + sd:.1f} s"}
+    if sq > 0:
+        single["quantize_gbs"] = round(bq / sq / 1e9, 4)
     procs = host_cores()
     out = {"value": single["value"], "unit": "GB/s", "cores": 1, "kind": "oracle",
            "kv_tokens_per_s": single["kv_tokens_per_s"],
-           "sample": f"{runs} x one batch row of {w.name} (quantize its full context + decode "
-                     f"all its query heads), single-threaded C oracle, {sq + sd:.1f} s",
+           "sample": f"{runs} x one batch row of {w.name} ({what_sample(w)}), "
+                     f"single-threaded C oracle, {sq + sd:.1f} s",
            "single_thread": single}
     if procs > 1:
         per_row = (sq + sd) / runs
@@ -623,9 +759,9 @@ def cpu_baseline(w, bits, budget_s):
             pool.close()
         out.update({"value": round((pb_q + pb_d) / wall / 1e9, 4), "cores": procs,
                     "kv_tokens_per_s": round(ptoks / wall, 1),
-                    "sample": f"{rows} x one batch row of {w.name} (quantize its full context "
-                              f"+ decode all its query heads), C oracle, one process per core "
-                              f"on {procs} cores, {wall:.1f} s wall"})
+                    "sample": f"{rows} x one batch row of {w.name} ({what_sample(w)}), C "
+                              f"oracle, one process per core on {procs} cores, {wall:.1f} s "
+                              f"wall"})
     return out
 
 
@@ -635,7 +771,7 @@ def run_reference(args):
     import oracle
     oracle.build()
     w = workloads.WORKLOADS[args.workload]
-    bits = w.bits[0]
+    bits = tuple(int(x) for x in args.bits.split(",")) if args.bits else default_bits(w)
     procs = host_cores()
     pool = OraclePool(procs, w, bits)
     try:
@@ -656,11 +792,11 @@ def run_reference(args):
         "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads,
                    "kv_heads": w.kv_heads, "head_dim": w.head_dim, "context": w.context,
                    "bits_k": bits[0], "bits_v": bits[1], "group": w.group,
-                   "step": f"{procs} batch rows of the workload per step, one per host core "
-                           "(bounded sample)"},
+                   "step": f"{procs} batch rows of the workload per step, one per host core, "
+                           f"each: {what_sample(w)} (bounded sample)"},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": procs, "kind": "oracle",
-                         "sample": f"{procs} batch rows per step, C oracle, one process per "
-                                   "core"},
+                         "sample": f"{procs} batch rows per step ({what_sample(w)}), C "
+                                   f"oracle, one process per core"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "kv_tokens_per_s": round(tot_t / tot_s, 1),
     }
@@ -672,12 +808,14 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama3_8b", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--bits", default=None, help="bits_k,bits_v (default: the workload's)")
     ap.add_argument("--rotate", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration kernel times after the timed region")
     ap.add_argument("--group-v", type=int, default=0,
                     help="values' group size (default: the workload's group)")
     ap.add_argument("--fused", action="store_true",

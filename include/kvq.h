@@ -315,6 +315,12 @@ int kvq_decode_attention(const kvq_cache_desc* cache, const void* q,
  * rows whose length is clamped (KVQ_DEVERR_SEQ_LEN) append nothing.  The
  * written bytes equal those of kvq_quantize_append() (same quantizer, same
  * format; positions outside the new range keep their bytes).
+ * When one kv head serves more query heads than one CTA takes (more than 8),
+ * every CTA of that kv head writes the new rows itself, without waiting for
+ * the others: the stores are whole 32-bit words (K codes, parameters) or
+ * 16-bit halves (V codes) carrying identical bits, so a copy that reads a
+ * row while another CTA stores it sees the same value either way.  Nothing
+ * else about the result depends on that ordering.
  */
 int kvq_append_decode_attention(const kvq_cache_desc* cache, const void* k_new,
                                 const void* v_new, int32_t in_dtype, int32_t n_new,
@@ -361,6 +367,21 @@ int kvq_decode_attention_static(const kvq_cache_desc* cache, const void* q,
  */
 int32_t kvq_decode_split_tokens(const kvq_cache_desc* cache,
                                 int32_t num_q_heads, int32_t max_seq_len);
+
+/*
+ * Failure-detection test knob; not for production use.  The summary page has
+ * no counterpart: it exists so that a test can make a bounded device wait run
+ * out without faulting or hanging the GPU.  With drop_stage >= 0, the next
+ * decode-attention launch in this process (only that one) arms stage
+ * `drop_stage` of the first warp's copy pipeline in its first CTA without
+ * issuing the copies, and every bounded wait of that launch gives up after
+ * wait_limit_ns (1000 .. 1e9 ns) instead of one second.  The wait on the
+ * dropped stage then runs out: the kernel flags KVQ_DEVERR_TIMEOUT, waits
+ * (bounded) for its copies in flight, and returns; that call's output is
+ * unspecified, and the cache is untouched.  drop_stage < 0 disarms the knob.
+ * Returns KVQ_OK, or KVQ_ERR_INVALID_ARG for a limit out of range.
+ */
+int kvq_debug_inject_wait_timeout(int32_t drop_stage, int64_t wait_limit_ns);
 
 /*
  * Reads and clears the current device's error word (bits of

@@ -93,6 +93,8 @@ def library() -> ctypes.CDLL:
     lib.kvq_device_error_flags.restype = ctypes.c_int
     lib.kvq_last_device_error.argtypes = [P]
     lib.kvq_last_device_error.restype = ctypes.c_int
+    lib.kvq_debug_inject_wait_timeout.argtypes = [I32, ctypes.c_int64]
+    lib.kvq_debug_inject_wait_timeout.restype = ctypes.c_int
     lib.kvq_strerror.argtypes = [I32]
     lib.kvq_strerror.restype = ctypes.c_char_p
     _lib = lib
@@ -273,6 +275,13 @@ def kvq_append_decode_attention(cache: KVCache, k_new: torch.Tensor, v_new: torc
         _DTYPE[out.dtype], ws_ptr, ws_bytes, _stream_ptr(stream))
     _check(st, "kvq_append_decode_attention")
     return out
+
+
+def kvq_debug_inject_wait_timeout(drop_stage: int, wait_limit_ns: int = 1_000_000) -> None:
+    """Test knob: the next decode launch drops one copy stage so that a bounded
+    wait runs out (see kvq.h); drop_stage < 0 disarms it."""
+    _check(library().kvq_debug_inject_wait_timeout(int(drop_stage), int(wait_limit_ns)),
+           "kvq_debug_inject_wait_timeout")
 
 
 def kvq_device_error_flags(stream: Optional[torch.cuda.Stream] = None) -> int:

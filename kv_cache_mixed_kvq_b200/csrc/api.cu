@@ -2,6 +2,7 @@
 // split-K plan, kernel selection and launches.  No allocation anywhere.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <map>
@@ -39,6 +40,11 @@ bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int groups_k, int g
 
 // Per-device error word (one copy on every device that loads the library).
 static __device__ uint32_t g_kvq_device_error;
+
+// Armed failure-detection test knob (kvq_debug_inject_wait_timeout): the
+// stage to drop in the next decode launch (-1: none) and its wait limit.
+static std::atomic<long long> g_fault_stage{-1};
+static std::atomic<long long> g_fault_limit_ns{0};
 
 namespace {
 
@@ -108,18 +114,21 @@ bool valid_dtype(int t) { return t == KVQ_F32 || t == KVQ_BF16 || t == KVQ_F16; 
 
 // Device address of the error word on the current device (looked up once per
 // device; the symbol's host-side name is not a device address).
+// Only a successful lookup is kept: a failed one is retried on the next call.
 int error_word(uint32_t** out) {
+  static std::mutex mu;
   static uint32_t* ptrs[kMaxDevices] = {};
-  static std::once_flag once[kMaxDevices];
-  static cudaError_t status[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
-  std::call_once(once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
     void* p = nullptr;
-    status[dev] = cudaGetSymbolAddress(&p, g_kvq_device_error);
+    if (cudaGetSymbolAddress(&p, g_kvq_device_error) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();  // reset the runtime's last-error state; the next call retries
+      return KVQ_ERR_CUDA;
+    }
     ptrs[dev] = static_cast<uint32_t*>(p);
-  });
-  if (status[dev] != cudaSuccess) return KVQ_ERR_CUDA;
+  }
   *out = ptrs[dev];
   return KVQ_OK;
 }
@@ -219,18 +228,21 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
   return KVQ_OK;
 }
 
-// Plans are cached per (device, shape, Hq, max_seq_len, split override):
-// the occupancy query behind a plan costs microseconds of host time.
+// Plans are cached per (device, shape incl. both group sizes and the flags,
+// Hq, max_seq_len, split override): the occupancy query behind a plan costs
+// microseconds of host time.  The plan never depends on the query type (the
+// workspace size is queried without it), so the occupancy of the 16-bit
+// query instance stands for every query type.
 int make_plan(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
-  using Key = std::tuple<int, int, int, int, int, int, int, int, int, int, long long>;
+  using Key = std::tuple<int, int, int, int, int, int, int, int, int, int, int, int, long long>;
   static std::mutex mu;
   static std::map<Key, Plan> cache;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
   long long override_split = 0;
   if (const char* env = std::getenv("KVQ_SPLIT_TOKENS")) override_split = std::atoll(env);
-  const Key key{dev, c->batch, c->kv_heads, c->head_dim, c->bits_k, c->bits_v, c->group, Hq,
-                max_seq_len, c->capacity, override_split};
+  const Key key{dev, c->batch, c->kv_heads, c->head_dim, c->bits_k, c->bits_v, c->group,
+                group_v_of(c), c->flags, Hq, max_seq_len, c->capacity, override_split};
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
@@ -381,6 +393,11 @@ int decode_impl(const kvq_cache_desc* cache, const void* k_new, const void* v_ne
     a.v_new = v_new;
     a.in_dtype = in_dtype;
     a.n_new = n_new;
+    // one-shot test knob: only the next launch after arming it carries it
+    const long long fault = g_fault_stage.exchange(-1);
+    a.fault_stage = fault >= 0 ? static_cast<int>(fault) : -1;
+    a.wait_limit_ns = fault >= 0 ? static_cast<unsigned long long>(g_fault_limit_ns.load())
+                                 : 1000000000ull;
     a.ws_o = ws_o;
     a.ws_lse = ws_lse;
     a.direct = p.direct;
@@ -432,6 +449,17 @@ int kvq_append_decode_attention(const kvq_cache_desc* cache, const void* k_new,
   return decode_impl(cache, n_new > 0 ? k_new : nullptr, n_new > 0 ? v_new : nullptr, in_dtype,
                      n_new, q, q_dtype, num_q_heads, seq_lens, max_seq_len, sm_scale, out,
                      out_dtype, workspace, workspace_bytes, stream);
+}
+
+int kvq_debug_inject_wait_timeout(int32_t drop_stage, int64_t wait_limit_ns) {
+  if (drop_stage < 0) {
+    g_fault_stage.store(-1);
+    return KVQ_OK;
+  }
+  if (wait_limit_ns < 1000 || wait_limit_ns > 1000000000LL) return KVQ_ERR_INVALID_ARG;
+  g_fault_limit_ns.store(wait_limit_ns);
+  g_fault_stage.store(drop_stage);
+  return KVQ_OK;
 }
 
 int kvq_device_error_flags(kvq_stream_t stream, uint32_t* flags) {

@@ -23,20 +23,23 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-// Device address of the scratch array on the current device.  The lookup is
-// made once per device, on the first call made with that device current.
+// Device address of the scratch array on the current device, looked up with
+// that device current.  A successful lookup is kept for the rest of the
+// process; a failed one returns KVQ_ERR_CUDA and is retried on the next call.
 int static_scratch(void** out) {
+  static std::mutex mu;
   static void* ptrs[kMaxDevices] = {};
-  static cudaError_t status[kMaxDevices] = {};
-  static std::once_flag once[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
-  std::call_once(once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
     void* p = nullptr;
-    status[dev] = cudaGetSymbolAddress(&p, g_kvq_static_scratch);
+    if (cudaGetSymbolAddress(&p, g_kvq_static_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return KVQ_ERR_CUDA;
+    }
     ptrs[dev] = p;
-  });
-  if (status[dev] != cudaSuccess || ptrs[dev] == nullptr) return KVQ_ERR_CUDA;
+  }
   *out = ptrs[dev];
   return KVQ_OK;
 }

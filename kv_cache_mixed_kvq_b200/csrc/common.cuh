@@ -116,15 +116,17 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// Longest a pipeline wait may take before the kernel gives up (1 s).
+// Longest a pipeline wait may take before the kernel gives up (1 s), unless
+// the launch carries a shorter limit (the failure-detection test knob).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
-// Slow path of mbar_wait_bounded: keep waiting, up to kWaitLimitNs.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* err) {
+// Slow path of mbar_wait_bounded: keep waiting, up to limit_ns.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                                   uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       flag_error(err, KVQ_DEVERR_TIMEOUT);
       return false;
     }
@@ -132,10 +134,11 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
 }
 
 // Bounded wait on an mbarrier phase: returns false (and flags
-// KVQ_DEVERR_TIMEOUT) if the phase did not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* err) {
+// KVQ_DEVERR_TIMEOUT) if the phase did not complete within limit_ns.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, err);
+  return mbar_wait_slow(bar, parity, err, limit_ns);
 }
 
 // Programmatic dependent launch.  pdl_wait() blocks until every grid this

@@ -312,6 +312,9 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     const uint32_t kbytes = n16 * C::KROW, vbytes = (n16 / 16) * C::VTILE;
     const uint32_t pkbytes = n16 * C::PROWK, pvbytes = n16 * C::PROWV;
     mbar_arrive_expect_tx(&wfull[sl], kbytes + vbytes + pkbytes + pvbytes);
+    if (it == a.fault_stage && warp == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
+        blockIdx.z == 0)
+      return;  // test knob: bytes announced, no copy issued (the wait runs out)
     bulk_copy_g2s(dst, a.k_codes + r * C::KROW, kbytes, &wfull[sl]);
     bulk_copy_g2s(dst + C::SLOT_K, a.v_codes + (r / 16) * C::VTILE, vbytes, &wfull[sl]);
     bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V,
@@ -807,7 +810,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       int next_page = 0;
       if (a.block_table != nullptr && lane == 0 && it + C::kSlots < my_iters)
         next_page = page_of(it + C::kSlots);
-      if (!mbar_wait_bounded(&wfull[sl], phase, err)) break;
+      if (!mbar_wait_bounded(&wfull[sl], phase, err, a.wait_limit_ns)) break;
       const uint8_t* st = wring + sl * C::SLOT_BYTES;
       const int base = it * C::kStageTokens + my_first;  // first position of this slot
       if (base + 16 * TPW <= n_tok) {
@@ -838,7 +841,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     // must land before shared memory is reused; bounded in any case.
     if (it < my_iters && lane == 0) {
       for (int k = it; k < min(my_iters, it + C::kSlots); ++k)
-        mbar_wait_bounded(&wfull[k % C::kSlots], (k / C::kSlots) & 1, err);
+        mbar_wait_bounded(&wfull[k % C::kSlots], (k / C::kSlots) & 1, err, a.wait_limit_ns);
     }
   }
 

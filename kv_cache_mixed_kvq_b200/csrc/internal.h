@@ -76,6 +76,12 @@ struct DecodeArgs {
   const void* k_new;
   const void* v_new;
   int in_dtype, n_new;
+  // Failure-detection test knob (kvq_debug_inject_wait_timeout): when
+  // fault_stage >= 0, the first CTA's first warp arms that stage of its copy
+  // pipeline without issuing its copies, so that the wait on it runs out;
+  // every bounded wait of the launch gives up after wait_limit_ns.
+  int fault_stage;
+  unsigned long long wait_limit_ns;
   float* ws_o;        // [B][Hq][num_splits][D] partial outputs
   float* ws_lse;      // [B][Hq][num_splits] log2-domain log-sum-exp
   uint32_t* err;

@@ -152,3 +152,10 @@ def test_fused_append_rejects_before_launch():
     assert call(dt=5) == kvq.KVQ_ERR_INVALID_ARG
     assert call(hq=7) == kvq.KVQ_ERR_INVALID_ARG         # decode checks still apply
     assert call(q=0) == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_wait_timeout_knob_is_validated_on_the_host():
+    lib = kvq.library()
+    assert lib.kvq_debug_inject_wait_timeout(0, 10) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_debug_inject_wait_timeout(0, 2_000_000_000) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_debug_inject_wait_timeout(-1, 0) == kvq.KVQ_OK

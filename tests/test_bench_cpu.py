@@ -89,22 +89,46 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert res["e2e"]["h2d_bytes_per_step"] == 0
 
 
-def test_cpu_baseline_uses_every_core_and_splits_the_phases():
+def test_cpu_baseline_uses_every_core():
     import bench
     w = bench.workloads.WORKLOADS["tiny"]
     res = bench.cpu_baseline(w, w.bits[0], 0.5)
     assert res["kind"] == "oracle" and res["value"] > 0
     assert res["cores"] == bench.host_cores()
     single = res["single_thread"]
-    assert single["cores"] == 1 and single["quantize_gbs"] > 0 and single["decode_gbs"] > 0
+    # the tiny step decodes a resident cache: only the decode is timed
+    assert single["cores"] == 1 and single["decode_gbs"] > 0 and "quantize_gbs" not in single
+
+
+def test_oracle_row_times_the_phases_of_the_step():
+    import bench
+    w = bench.workloads.WORKLOADS["llama3_8b"]  # its step quantizes the full cache
+    tq, td, bq, bd, toks = bench.OracleRow(w, (4, 2), 0, seed=0).run()
+    assert tq > 0 and td > 0 and toks == 4096
+    assert (bq, bd) == bench.row_bytes(w, (4, 2), 4096)
+    # one row's share of the whole step's algorithmic bytes
+    nb = bench.algorithmic_bytes(w, (4, 2), 4096, [4096] * 8)
+    assert bq * 8 == nb["quantize"] and bd * 8 == nb["decode"]
+    w = bench.workloads.WORKLOADS["ragged"]  # decode only, over a quantized row
+    row = bench.OracleRow(w, (4, 2), 5, seed=1)
+    assert row.length == int(bench.workloads.seq_lens(w)[5]) and row.hc is not None
 
 
 def test_rotation_exceeds_twice_the_l2():
     import bench
+    l2 = 126 * 2**20
     for step_bytes in (1e3, 29.4e6, 118e6, 193e6, 248e6, 1e9):
-        n = bench.sets_needed(step_bytes, 3)
+        n = bench.sets_needed(step_bytes, 3, l2)
         assert 3 <= n <= bench.MAX_SETS
         if n < bench.MAX_SETS:
-            assert (n - 1) * step_bytes >= 2 * bench.L2_BYTES
-    assert bench.sets_needed(193e6, 3) == 3      # the default workload keeps three sets
-    assert bench.sets_needed(29.4e6, 3) == 10
+            assert (n - 1) * step_bytes >= 2 * l2
+    assert bench.sets_needed(248e6, 3, l2) == 3      # the ragged step keeps three sets
+    assert bench.sets_needed(29.4e6, 3, l2) == 10
+
+
+def test_config_sweep_covers_every_workload_and_bit_pair():
+    import bench
+    got = {(n, b) for n, b in bench.CONFIG_SWEEP}
+    want = {(n, b) for n, w in bench.workloads.WORKLOADS.items() for b in w.bits}
+    assert got == want
+    assert bench.DEFAULT_WORKLOAD == "ragged" and bench.KERNEL_REPS >= 50

@@ -4,9 +4,11 @@ For callers that may not allocate device memory (engines that plan all
 device memory up front, plain-C hosts without an allocator), the library
 offers a variant whose split-K scratch is a fixed array in its device image.
 This file is collected last on purpose.  It calls the variant through the C
-ABI twice in a row with different inputs and checks each output against the
-regular entry point's within the attention tolerance of the other tests; it
-also checks that a shape needing more than the fixed scratch is refused.
+ABI on a large multi-split shape and then twice in a row on a smaller one
+(stale partials of another plan are left in the scratch), and checks that
+each output equals the regular entry point's bit for bit: both run the same
+split plan and the same deterministic kernels.  It also checks that a shape
+needing more than the fixed scratch is refused.
 """
 import ctypes
 
@@ -14,7 +16,6 @@ import pytest
 import torch
 
 import kv_cache_mixed_kvq_b200 as kvq
-from tests.gpu_util import TOL
 
 pytestmark = pytest.mark.gpu
 
@@ -40,24 +41,43 @@ def _filled_cache(B, Hkv, D, T, seed):
     return cache
 
 
+def _static_vs_regular(fn, cache, Hq, lens, T, seed):
+    """One call of each entry point on the same inputs; the static one must
+    reproduce the regular one bit for bit (same plan, same kernels)."""
+    B, D = cache.batch, cache.head_dim
+    q = torch.randn(B, Hq, D, generator=torch.Generator().manual_seed(seed)).to(
+        torch.bfloat16).cuda()
+    ref = kvq.kvq_decode_attention(cache, q, lens, T, out_dtype=torch.float32)
+    out = torch.full((B, Hq, D), float("nan"), dtype=torch.float32, device="cuda")
+    desc = cache.desc()
+    st = fn(ctypes.byref(desc), q.data_ptr(), kvq.KVQ_BF16, Hq, lens.data_ptr(), T, 0.0,
+            out.data_ptr(), kvq.KVQ_F32, torch.cuda.current_stream().cuda_stream)
+    assert st == kvq.KVQ_OK, kvq.kvq_strerror(st)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    assert torch.equal(out, ref), f"max difference {(out - ref).abs().max().item():.3e}"
+    return ref
+
+
 def test_static_matches_regular_twice():
     fn = _static_fn()
+    # A larger shape first, so that the second, smaller call finds the
+    # scratch holding stale partials of a different split plan.
+    big = _filled_cache(8, 8, 128, 4096, seed=2)
+    lens_big = torch.full((8,), 4096, dtype=torch.int32, device="cuda")
+    ws_big = kvq.kvq_decode_workspace_bytes(big, 32, 4096)
+    assert 0 < ws_big <= STATIC_BYTES
+    assert kvq.kvq_decode_split_tokens(big, 32, 4096) < 4096  # several splits per row
+    _static_vs_regular(fn, big, 32, lens_big, 4096, seed=7)
+
     B, Hkv, Hq, D, T = 4, 8, 32, 128, 3000
     cache = _filled_cache(B, Hkv, D, T, seed=1)
     lens = torch.tensor([3000, 1, 1777, 64], dtype=torch.int32, device="cuda")
-    stream = torch.cuda.current_stream()
-    for call in range(2):
-        q = torch.randn(B, Hq, D, generator=torch.Generator().manual_seed(10 + call)).to(
-            torch.bfloat16).cuda()
-        ref = kvq.kvq_decode_attention(cache, q, lens, T, out_dtype=torch.float32)
-        out = torch.full((B, Hq, D), float("nan"), dtype=torch.float32, device="cuda")
-        desc = cache.desc()
-        st = fn(ctypes.byref(desc), q.data_ptr(), kvq.KVQ_BF16, Hq, lens.data_ptr(), T, 0.0,
-                out.data_ptr(), kvq.KVQ_F32, stream.cuda_stream)
-        assert st == kvq.KVQ_OK, kvq.kvq_strerror(st)
-        torch.cuda.synchronize()
-        assert torch.isfinite(out).all()
-        assert (out - ref).abs().max().item() <= TOL
+    ws = kvq.kvq_decode_workspace_bytes(cache, Hq, T)
+    assert 0 < ws < ws_big  # this shape uses the scratch too, with another plan
+    assert kvq.kvq_decode_split_tokens(cache, Hq, T) < T
+    outs = [_static_vs_regular(fn, cache, Hq, lens, T, seed=10 + call) for call in range(2)]
+    assert not torch.equal(outs[0], outs[1])  # the two calls had different queries
     assert kvq.kvq_device_error_flags() == 0
 
 
