@@ -8,6 +8,7 @@
 #include <map>
 #include <mutex>
 #include <set>
+#include <string>
 #include <tuple>
 #include <utility>
 
@@ -23,6 +24,29 @@ bool get_decode_kernel_k4v8(int, int, int, int, DecodeKernel*);
 bool get_decode_kernel_k8v2(int, int, int, int, DecodeKernel*);
 bool get_decode_kernel_k8v4(int, int, int, int, DecodeKernel*);
 bool get_decode_kernel_k8v8(int, int, int, int, DecodeKernel*);
+
+bool get_decode_tc_kernel_k2v2(int, int, int, DecodeKernel*);
+bool get_decode_tc_kernel_k2v4(int, int, int, DecodeKernel*);
+bool get_decode_tc_kernel_k2v8(int, int, int, DecodeKernel*);
+bool get_decode_tc_kernel_k4v2(int, int, int, DecodeKernel*);
+bool get_decode_tc_kernel_k4v4(int, int, int, DecodeKernel*);
+bool get_decode_tc_kernel_k4v8(int, int, int, DecodeKernel*);
+bool get_decode_tc_kernel_k8v2(int, int, int, DecodeKernel*);
+bool get_decode_tc_kernel_k8v4(int, int, int, DecodeKernel*);
+bool get_decode_tc_kernel_k8v8(int, int, int, DecodeKernel*);
+
+bool get_decode_tc_kernel(int bits_k, int bits_v, int groups_k, int groups_v, int heads_per_cta,
+                          DecodeKernel* out) {
+  using Fn = bool (*)(int, int, int, DecodeKernel*);
+  static const Fn table[3][3] = {
+      {get_decode_tc_kernel_k2v2, get_decode_tc_kernel_k2v4, get_decode_tc_kernel_k2v8},
+      {get_decode_tc_kernel_k4v2, get_decode_tc_kernel_k4v4, get_decode_tc_kernel_k4v8},
+      {get_decode_tc_kernel_k8v2, get_decode_tc_kernel_k8v4, get_decode_tc_kernel_k8v8}};
+  auto idx = [](int b) { return b == 2 ? 0 : b == 4 ? 1 : b == 8 ? 2 : -1; };
+  const int i = idx(bits_k), j = idx(bits_v);
+  if (i < 0 || j < 0) return false;
+  return table[i][j](groups_k, groups_v, heads_per_cta, out);
+}
 
 bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int groups_k, int groups_v,
                        int variant, DecodeKernel* out) {
@@ -133,6 +157,29 @@ int error_word(uint32_t** out) {
   return KVQ_OK;
 }
 
+int variant_of(int heads_per_cta, int q_dtype);
+
+// Which decode kernel runs.  The register-fragment kernel (mma.sync, codes
+// unpacked straight into tensor-core fragments) serves every shape.  The
+// tensor-memory kernel (tcgen05, head_dim 128, no fused append) is selected
+// with KVQ_DECODE_KERNEL=tcgen05; it computes the same result but measured
+// slower on B200 (its small-N products are bound by the tensor core reading
+// the unpacked binary16 operands, about 75 cycles per 128x16x16 product).
+bool use_tc_kernel(const kvq_cache_desc* c, bool fused) {
+  if (c->head_dim != 128 || fused) return false;
+  const char* env = std::getenv("KVQ_DECODE_KERNEL");
+  return env && std::string(env) == "tcgen05";
+}
+
+bool select_decode_kernel(const kvq_cache_desc* c, int heads_per_cta, int q_dtype, bool fused,
+                          DecodeKernel* k) {
+  const int gk = c->head_dim / c->group, gv = c->head_dim / group_v_of(c);
+  if (use_tc_kernel(c, fused))
+    return kvq::get_decode_tc_kernel(c->bits_k, c->bits_v, gk, gv, heads_per_cta, k);
+  return kvq::get_decode_kernel(c->head_dim, c->bits_k, c->bits_v, gk, gv,
+                                variant_of(heads_per_cta, q_dtype), k);
+}
+
 // Opt a kernel in to more than 48 KB of dynamic shared memory, once per
 // (device, kernel).
 cudaError_t prepare_kernel(const DecodeKernel& k) {
@@ -144,7 +191,15 @@ cudaError_t prepare_kernel(const DecodeKernel& k) {
   std::lock_guard<std::mutex> lock(mu);
   if (done.count({dev, k.fn})) return cudaSuccess;
   e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem_bytes);
+  // the largest shared-memory carveout, so that the occupancy the plan is
+  // sized for (several CTAs per SM) is the one the hardware gives
   if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k.fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess && k.fn_fused != nullptr)
+    e = cudaFuncSetAttribute(k.fn_fused, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess && k.fn_fused != nullptr)
     e = cudaFuncSetAttribute(k.fn_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              k.smem_bytes);
   if (e == cudaSuccess) done.insert({dev, k.fn});
@@ -183,11 +238,10 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
     p->ws_bytes = 0;
     return KVQ_OK;
   }
+  // the plan is that of the kernel a plain decode runs (the fused append
+  // follows the same plan, so that the workspace size does not depend on it)
   DecodeKernel k;
-  if (!kvq::get_decode_kernel(c->head_dim, c->bits_k, c->bits_v, c->head_dim / c->group,
-                              c->head_dim / group_v_of(c),
-                              variant_of(p->heads_per_cta, KVQ_BF16), &k))
-    return KVQ_ERR_UNSUPPORTED;
+  if (!select_decode_kernel(c, p->heads_per_cta, KVQ_BF16, false, &k)) return KVQ_ERR_UNSUPPORTED;
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -196,20 +250,22 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.fn, k.threads, k.smem_bytes) !=
           cudaSuccess)
     return KVQ_ERR_CUDA;
+  if (k.max_per_sm > 0 && per_sm > k.max_per_sm) per_sm = k.max_per_sm;
   if (per_sm < 1) per_sm = 1;
   const long long units = static_cast<long long>(c->batch) * c->kv_heads * p->head_groups;
   const long long slots = static_cast<long long>(sms) * per_sm;
-  const long long max64 = (max_seq_len + 63LL) / 64 * 64;
+  const long long T = k.tile;  // splits are whole tiles of the kernel
+  const long long max_t = (max_seq_len + T - 1) / T * T;
   long long split;
   if (slots >= 4 * units) {
     const long long per_unit = slots / units;
-    split = ((max_seq_len + per_unit - 1) / per_unit + 63) / 64 * 64;
+    split = ((max_seq_len + per_unit - 1) / per_unit + T - 1) / T * T;
   } else {
     const long long work = units * max_seq_len;
-    split = ((work + 3 * slots - 1) / (3 * slots) + 63) / 64 * 64;
+    split = ((work + 3 * slots - 1) / (3 * slots) + T - 1) / T * T;
   }
   if (split < 256) split = 256;
-  if (split > max64) split = max64;
+  if (split > max_t) split = max_t;
   if (const char* env = std::getenv("KVQ_SPLIT_TOKENS")) {
     const long long v = std::atoll(env);
     if (v >= 64 && v % 64 == 0) split = v;
@@ -242,7 +298,8 @@ int make_plan(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
   long long override_split = 0;
   if (const char* env = std::getenv("KVQ_SPLIT_TOKENS")) override_split = std::atoll(env);
   const Key key{dev, c->batch, c->kv_heads, c->head_dim, c->bits_k, c->bits_v, c->group,
-                group_v_of(c), c->flags, Hq, max_seq_len, c->capacity, override_split};
+                group_v_of(c), (c->flags << 1) | (use_tc_kernel(c, false) ? 1 : 0), Hq,
+                max_seq_len, c->capacity, override_split};
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
@@ -363,9 +420,7 @@ int decode_impl(const kvq_cache_desc* cache, const void* k_new, const void* v_ne
   float* ws_lse = ws_o ? ws_o + p.ws_o_floats : nullptr;
   if (p.num_splits > 0) {
     DecodeKernel k;
-    if (!kvq::get_decode_kernel(D, cache->bits_k, cache->bits_v, D / cache->group,
-                                D / group_v_of(cache),
-                                variant_of(p.heads_per_cta, q_dtype), &k))
+    if (!select_decode_kernel(cache, p.heads_per_cta, q_dtype, k_new != nullptr, &k))
       return KVQ_ERR_UNSUPPORTED;
     if (prepare_kernel(k) != cudaSuccess) return KVQ_ERR_CUDA;
     kvq::DecodeArgs a;

@@ -60,6 +60,16 @@ __device__ __forceinline__ float load_elem(const void* base, int dtype, size_t i
   return __half2float(__ushort_as_half(u));
 }
 
+// One attention output element in the caller's type.
+__device__ __forceinline__ void store_out(void* out, int dtype, size_t i, float v) {
+  if (dtype == KVQ_F32)
+    reinterpret_cast<float*>(out)[i] = v;
+  else if (dtype == KVQ_BF16)
+    reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<__half*>(out)[i] = __float2half_rn(v);
+}
+
 // --------------------------------------------------------------- error word
 __device__ __forceinline__ void flag_error(uint32_t* err, uint32_t bits) {
   if (err) atomicOr(err, bits);

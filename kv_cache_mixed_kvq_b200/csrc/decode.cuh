@@ -208,16 +208,6 @@ __device__ __forceinline__ void lds_param_pair(const uint32_t* p, uint32_t (&w0)
   }
 }
 
-// One attention output element in the caller's type.
-__device__ __forceinline__ void store_out(void* out, int dtype, size_t i, float v) {
-  if (dtype == KVQ_F32)
-    reinterpret_cast<float*>(out)[i] = v;
-  else if (dtype == KVQ_BF16)
-    reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
-  else
-    reinterpret_cast<__half*>(out)[i] = __float2half_rn(v);
-}
-
 // FUSED: the instance used by the fused append + decode call (the append
 // prologue is compiled only there, so the plain decode keeps its registers
 // and schedule).
@@ -941,6 +931,8 @@ DecodeKernel make_decode_kernel() {
   k.smem_bytes = C::SMEM_BYTES;
   k.launch = &launch_decode<C, false>;
   k.launch_fused = &launch_decode<C, true>;
+  k.tile = 64;
+  k.max_per_sm = 0;
   return k;
 }
 

@@ -100,6 +100,8 @@ struct DecodeKernel {
   const void* fn_fused;  // the same with the fused append (k_new != NULL)
   int threads;
   int smem_bytes;
+  int tile;              // split lengths are rounded to a multiple of this
+  int max_per_sm;        // CTAs per SM the kernel allows itself (0: no limit of its own)
   cudaError_t (*launch)(const DecodeArgs&, dim3 grid, cudaStream_t stream);
   cudaError_t (*launch_fused)(const DecodeArgs&, dim3 grid, cudaStream_t stream);
 };
@@ -107,6 +109,11 @@ struct DecodeKernel {
 // Returns false if (D, bits, key groups, value groups, variant) has no instance.
 bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int groups_k, int groups_v,
                        int variant, DecodeKernel* out);
+
+// The tensor-memory decode kernel (head_dim 128, no fused append): false if
+// (bits, key groups, value groups) has no instance.
+bool get_decode_tc_kernel(int bits_k, int bits_v, int groups_k, int groups_v, int heads_per_cta,
+                          DecodeKernel* out);
 
 struct CombineArgs {
   const float* ws_o;
