@@ -210,8 +210,17 @@ struct Plan {
   int heads_per_cta, head_groups, split_tokens, num_splits;
   bool direct;         // one split per row: the decode writes the output itself
   size_t ws_o_floats;  // partial outputs [B][Hq][splits][D]
-  size_t ws_bytes;     // partials + log-sum-exps
+  size_t ws_bytes;     // partials + log-sum-exps (enough for either schedule)
+  // Balanced (stream-K) schedule of a plain decode (stream_q > 0): a one-wave
+  // grid of stream_grid CTAs, each taking at least stream_q stages;
+  // stream_parts partial slots per row.
+  int stream_q, stream_grid, stream_parts, stage_tokens;
+  size_t stream_o_floats;
 };
+
+// Smallest share of stages of a CTA in the balanced schedule (it bounds the
+// partial results a unit can leave, hence the workspace).
+constexpr int kStreamMinStages = 4;
 
 int variant_of(int heads_per_cta, int q_dtype) {
   return (heads_per_cta <= 4 ? 0 : 2) + (q_dtype == KVQ_F32 ? 1 : 0);
@@ -281,6 +290,30 @@ int make_plan_uncached(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p
     p->ws_bytes = static_cast<size_t>(c->batch) * Hq * p->num_splits * (c->head_dim + 1) * 4;
     p->ws_bytes = (p->ws_bytes + 15) / 16 * 16;
   }
+  // Balanced schedule (KVQ_DECODE_SCHEDULE=balanced), when rows need
+  // splitting anyway and the batch fits the kernel's row table: one wave of
+  // CTAs with equal shares of stages.  Not the default: measured on B200, a
+  // span costs about as much as four stages of fixed work, and SMs of
+  // different GPCs stream at speeds up to ~15% apart, so a static partition
+  // ends later than the block scheduler's dynamic one on the ragged batch.
+  p->stream_q = 0;
+  p->stream_grid = 0;
+  p->stream_parts = 0;
+  p->stage_tokens = k.stage_tokens;
+  p->stream_o_floats = 0;
+  const char* sched = std::getenv("KVQ_DECODE_SCHEDULE");
+  const bool stream_ok = sched && std::string(sched) == "balanced" &&
+                         std::getenv("KVQ_SPLIT_TOKENS") == nullptr;
+  if (stream_ok && !p->direct && k.stage_tokens > 0 && c->batch <= kvq::kStreamRows) {
+    const long long ns_max = (max_seq_len + k.stage_tokens - 1) / k.stage_tokens;
+    p->stream_q = kStreamMinStages;
+    p->stream_grid = static_cast<int>(slots);
+    p->stream_parts = static_cast<int>((ns_max + kStreamMinStages - 1) / kStreamMinStages + 1);
+    p->stream_o_floats = static_cast<size_t>(c->batch) * Hq * p->stream_parts * c->head_dim;
+    size_t sb = static_cast<size_t>(c->batch) * Hq * p->stream_parts * (c->head_dim + 1) * 4;
+    sb = (sb + 15) / 16 * 16;
+    if (sb > p->ws_bytes) p->ws_bytes = sb;
+  }
   return KVQ_OK;
 }
 
@@ -297,6 +330,8 @@ int make_plan(const kvq_cache_desc* c, int Hq, int max_seq_len, Plan* p) {
   if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
   long long override_split = 0;
   if (const char* env = std::getenv("KVQ_SPLIT_TOKENS")) override_split = std::atoll(env);
+  if (const char* env = std::getenv("KVQ_DECODE_SCHEDULE"))
+    if (std::string(env) == "balanced") override_split = -1 - override_split;
   const Key key{dev, c->batch, c->kv_heads, c->head_dim, c->bits_k, c->bits_v, c->group,
                 group_v_of(c), (c->flags << 1) | (use_tc_kernel(c, false) ? 1 : 0), Hq,
                 max_seq_len, c->capacity, override_split};
@@ -417,11 +452,15 @@ int decode_impl(const kvq_cache_desc* cache, const void* k_new, const void* v_ne
   const int D = cache->head_dim;
   const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf(static_cast<float>(D));
   float* ws_o = p.ws_bytes > 0 ? static_cast<float*>(workspace) : nullptr;
-  float* ws_lse = ws_o ? ws_o + p.ws_o_floats : nullptr;
+  float* ws_lse = nullptr;
+  bool balanced = false;  // the balanced (stream-K) schedule runs
   if (p.num_splits > 0) {
     DecodeKernel k;
     if (!select_decode_kernel(cache, p.heads_per_cta, q_dtype, k_new != nullptr, &k))
       return KVQ_ERR_UNSUPPORTED;
+    // the balanced schedule serves the kernel it was planned for (both the
+    // plain and the fused decode, so that they take the same splits)
+    balanced = p.stream_q > 0 && k.stage_tokens == p.stage_tokens;
     if (prepare_kernel(k) != cudaSuccess) return KVQ_ERR_CUDA;
     kvq::DecodeArgs a;
     a.k_codes = cache->k_codes;
@@ -440,7 +479,9 @@ int decode_impl(const kvq_cache_desc* cache, const void* k_new, const void* v_ne
     a.heads_per_cta = p.heads_per_cta;
     a.head_groups = p.head_groups;
     a.split_tokens = p.split_tokens;
-    a.num_splits = p.num_splits;
+    a.num_splits = balanced ? p.stream_parts : p.num_splits;
+    a.stream_q = balanced ? p.stream_q : 0;
+    ws_lse = ws_o ? ws_o + (balanced ? p.stream_o_floats : p.ws_o_floats) : nullptr;
     a.sm_scale_log2 = scale * 1.4426950408889634f;
     a.rotate_q = (cache->flags & KVQ_FLAG_ROTATE_KEYS) != 0;
     page_args(cache, &a.block_table, &a.page_shift, &a.pages_per_seq, &a.num_pages);
@@ -455,15 +496,16 @@ int decode_impl(const kvq_cache_desc* cache, const void* k_new, const void* v_ne
                                  : 1000000000ull;
     a.ws_o = ws_o;
     a.ws_lse = ws_lse;
-    a.direct = p.direct;
+    a.direct = p.direct && !balanced;
     a.out = out;
     a.out_dtype = out_dtype;
     st = error_word(&a.err);
     if (st != KVQ_OK) return st;
-    const dim3 grid(p.num_splits, cache->kv_heads * p.head_groups, cache->batch);
+    const dim3 grid = balanced ? dim3(p.stream_grid, 1, 1)
+                             : dim3(p.num_splits, cache->kv_heads * p.head_groups, cache->batch);
     if ((k_new != nullptr ? k.launch_fused : k.launch)(a, grid, s) != cudaSuccess)
       return KVQ_ERR_CUDA;
-    if (p.direct) return KVQ_OK;
+    if (a.direct) return KVQ_OK;
   }
   kvq::CombineArgs ca;
   ca.ws_o = ws_o;
@@ -477,7 +519,14 @@ int decode_impl(const kvq_cache_desc* cache, const void* k_new, const void* v_ne
   ca.capacity = cache->capacity;
   ca.max_seq_len = max_seq_len;
   ca.split_tokens = p.split_tokens;
-  ca.num_splits = p.num_splits;
+  ca.num_splits = balanced ? p.stream_parts : p.num_splits;
+  ca.stream_q = balanced ? p.stream_q : 0;
+  ca.stream_grid = p.stream_grid;
+  ca.stage_tokens = p.stage_tokens;
+  ca.kv_heads = cache->kv_heads;
+  ca.head_groups = p.head_groups;
+  ca.gq = num_q_heads / cache->kv_heads;
+  ca.heads_per_cta = p.heads_per_cta;
   return to_status(kvq::launch_combine(ca, s));
 }
 }  // namespace

@@ -5,7 +5,8 @@
 //   o = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L),   L = max_s lse_s.
 // One CTA of four warps per (batch row, query head); the warps take every
 // fourth split, each lane owns D/32 elements, and the warps' results are
-// merged through shared memory.
+// merged through shared memory.  With the decode's balanced schedule the
+// partials of a row are those of the CTAs that covered its unit.
 #include "common.cuh"
 #include "internal.h"
 
@@ -21,17 +22,45 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
   const int row = blockIdx.x;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  pdl_wait();
-  pdl_trigger();
   const int b = row / a.q_heads;
-  int len = a.seq_lens[b];
-  len = max(0, min(len, min(a.max_seq_len, a.capacity)));
-  const int ns = (len + a.split_tokens - 1) / a.split_tokens;
+  const int lim = min(a.max_seq_len, a.capacity);
+  int ns;  // partial results of this row
+  if (a.stream_q > 0) {
+    // balanced schedule: the CTAs that covered this row's unit, from the same
+    // prefix sums as the decode kernel (built from the lengths alone, before
+    // the wait for the decode grid); a unit one CTA covered whole was written
+    // by it directly
+    __shared__ int s_off[kStreamRows + 1];
+    __shared__ int s_w[4];
+    const int units = a.kv_heads * a.head_groups;  // per row
+    stream_row_offsets(a.seq_lens, a.batch, lim, units, a.stage_tokens, s_off, nullptr, s_w);
+    pdl_wait();
+    pdl_trigger();
+    const int S = s_off[kStreamRows];
+    const int Q = max(a.stream_q, (S + a.stream_grid - 1) / a.stream_grid);
+    const int hq = row % a.q_heads;
+    const int u = (hq / a.gq) * a.head_groups + (hq % a.gq) / a.heads_per_cta;
+    const int nsu = (s_off[b + 1] - s_off[b]) / units;
+    ns = 0;
+    if (nsu > 0) {
+      const int ubase = s_off[b] + u * nsu;
+      ns = (ubase + nsu - 1) / Q - ubase / Q + 1;
+      if (ns == 1) return;
+    }
+  } else {
+    // (the lengths are read before the wait: no kernel of this library
+    // writes them)
+    const int len = max(0, min(a.seq_lens[b], lim));
+    ns = (len + a.split_tokens - 1) / a.split_tokens;
+    pdl_wait();
+    pdl_trigger();
+  }
   const size_t base = static_cast<size_t>(row) * a.num_splits;
 
   // Warp w merges splits w, w+4, w+8, ... with its own running maximum M;
-  // lanes load 32 of its log-sum-exps at a time, then the partial outputs of
-  // U splits at a time are all requested before any is used.
+  // lanes load 32 of its log-sum-exps at a time; the partial outputs of U
+  // splits at a time are all requested before any is used (the first U
+  // together with the log-sum-exps).
   float M = -INFINITY, den = 0.0f;
   float acc[PER];
 #pragma unroll
@@ -39,19 +68,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
   const int mine = ns > warp ? (ns - warp + 3) / 4 : 0;  // splits of this warp
   for (int c0 = 0; c0 < mine; c0 += 32) {
     const int cnt = min(32, mine - c0);
-    const float lse = lane < cnt ? a.ws_lse[base + warp + 4 * (c0 + lane)] : -INFINITY;
-    float cm = lse;
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, m));
-    const float Mn = fmaxf(M, cm);
-    const float r = exp2_approx(M - Mn);  // M = -inf on the first chunk: r = 0
-    den *= r;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] *= r;
-    M = Mn;
-    const float wl = lane < cnt ? exp2_approx(lse - M) : 0.0f;
-    for (int s = 0; s < cnt; s += U) {
-      float v[U][PER];
+    float v[U][PER];
+    auto load = [&](int s) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int si = warp + 4 * (c0 + min(s + u, cnt - 1));
@@ -64,6 +82,21 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
           v[u][0] = t.x; v[u][1] = t.y;
         }
       }
+    };
+    load(0);
+    const float lse = lane < cnt ? a.ws_lse[base + warp + 4 * (c0 + lane)] : -INFINITY;
+    float cm = lse;
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, m));
+    const float Mn = fmaxf(M, cm);
+    const float r = exp2_approx(M - Mn);  // M = -inf on the first chunk: r = 0
+    den *= r;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] *= r;
+    M = Mn;
+    const float wl = lane < cnt ? exp2_approx(lse - M) : 0.0f;
+    for (int s = 0; s < cnt; s += U) {
+      if (s > 0) load(s);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const float w = __shfl_sync(0xffffffffu, wl, (s + u) & 31);

@@ -5,6 +5,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "internal.h"
 #include "kvq.h"
 
 namespace kvq {
@@ -73,6 +74,47 @@ __device__ __forceinline__ void store_out(void* out, int dtype, size_t i, float 
 // --------------------------------------------------------------- error word
 __device__ __forceinline__ void flag_error(uint32_t* err, uint32_t bits) {
   if (err) atomicOr(err, bits);
+}
+
+// ------------------------------------------------ balanced decode schedule
+// off[r] = units * sum_{r' < r} ceil(len_r' / T) for r = 0 .. kStreamRows,
+// with each length clamped to [0, lim] (rows past `batch` count nothing);
+// lens (when not NULL): the raw lengths, kStreamRows entries (0 past
+// `batch`).  Reads only the lengths, so it may run before the wait for the
+// previous grid.  Called by all 128 threads of the CTA; wsum: 4 ints of
+// shared scratch.  Ends with a CTA barrier.
+__device__ __forceinline__ void stream_row_offsets(const int32_t* seq_lens, int batch, int lim,
+                                                   int units, int T, int* off, int* lens,
+                                                   int* wsum) {
+  constexpr int R = kStreamRows / 128;
+  int cnt[R], tot = 0;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int r = R * threadIdx.x + i;
+    const int raw = r < batch ? seq_lens[r] : 0;
+    if (lens != nullptr) lens[r] = raw;
+    const int len = max(0, min(raw, lim));
+    cnt[i] = units * ((len + T - 1) / T);
+    tot += cnt[i];
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = tot;  // inclusive scan of the threads' totals within the warp
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, m);
+    if (lane >= m) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int before = incl - tot;
+  for (int w = 0; w < warp; ++w) before += wsum[w];
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    off[R * threadIdx.x + i] = before;
+    before += cnt[i];
+  }
+  if (threadIdx.x == 127) off[kStreamRows] = before;
+  __syncthreads();
 }
 
 // ------------------------------------------------- mbarrier / bulk copies

@@ -54,6 +54,10 @@ struct DecodeCfg {
   static constexpr int D = D_, BK = BK_, BV = BV_, QS = QS_, NQ = NQ_, NP = NP_;
   static constexpr int NGK = NGK_, NGV = NGV_;
   static constexpr int kWarps = 4;  // warps per CTA; each runs its own copy pipeline
+  // CTAs per SM the registers must allow: four for up to four heads per CTA,
+  // three for 5..8 heads with 16-bit queries (two with 32-element key
+  // groups), two with binary32 queries
+  static constexpr int kMinBlocks = NP_ == 1 ? 4 : (QS_ == 1 && NGK_ < 4) ? 3 : 2;
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int TPW = 2;     // 16-token tiles per warp per stage
   static constexpr int kStageTokens = 16 * TPW * kWarps;
@@ -82,12 +86,29 @@ struct DecodeCfg {
   static constexpr int WB_RS = 24;  // halves per row: 16 positions + pad (conflict-free)
   static constexpr int WB_HALVES = NGV * 8 * 2 * WB_RS;
   static constexpr int WB_BYTES = TPW * kWarps * WB_HALVES * 2;
+  // the warps' partial outputs at the end of a span, [warp][head][D] binary32,
+  // share the staging buffer's region (the ring keeps receiving the next
+  // span's copies meanwhile)
+  static constexpr int OB_HEADS = 4 * NP;
+  static constexpr int OB_BYTES = kWarps * OB_HEADS * D * 4;
+  static constexpr int STAGE_BYTES = WB_BYTES > OB_BYTES ? WB_BYTES : OB_BYTES;
+  // query rows of a span ([head][D] in the query type, binary32 at most),
+  // two buffers: the next span's rows arrive while this span runs
+  static constexpr int QBUF_BYTES = OB_HEADS * D * 4;
   static constexpr int ALPHA_FLOATS = kWarps * 8;
   static constexpr int MERGE_FLOATS = kWarps * 8 * (2 + NGV) + 2 * 8 * (kWarps + 1);
-  static constexpr int SMEM_BYTES =
-      RING_BYTES + WB_BYTES + 4 * (ALPHA_FLOATS + MERGE_FLOATS) + 8 * kWarps * kSlots;
+  static constexpr int QBUF_OFF = RING_BYTES + STAGE_BYTES;
+  static constexpr int ALPHA_OFF = QBUF_OFF + 2 * QBUF_BYTES;
+  // mbarriers: [warp][slot] copy slots, then the two query buffers; then
+  // the CTA's span counter and query flag (4 ints) and each warp's view of
+  // the next span (4 ints per warp)
+  static constexpr int BAR_OFF = ALPHA_OFF + 4 * (ALPHA_FLOATS + MERGE_FLOATS);
+  static constexpr int CTL_OFF = BAR_OFF + 8 * (kWarps * kSlots + 2);
+  // + the balanced schedule's row table: lengths (kStreamRows ints) and the
+  // prefix sums of the rows' stages (kStreamRows + 1 ints)
+  static constexpr int SMEM_BYTES = CTL_OFF + 16 + 16 * kWarps + 4 * (2 * kStreamRows + 1);
   static constexpr int HT = QS == 1 ? 2 * NQ : NQ;  // score head slots per lane
-  static_assert(RING_BYTES >= kWarps * 8 * D * 4, "merge buffer must fit in the ring");
+  static_assert(kThreads == 128, "the stream schedule's scan runs on 128 threads");
   static_assert(WB_BYTES >= 8 * D * 4, "rotated queries must fit in the staging buffer");
   // fused append: rows whose inputs one warp loads before quantizing them,
   // and its shared scratch (one binary32 row and one row of codes)
@@ -95,6 +116,7 @@ struct DecodeCfg {
   static constexpr int APPEND_SCRATCH = 5 * D;
   static_assert(WB_BYTES >= kWarps * APPEND_SCRATCH, "append scratch must fit in the staging buffer");
   static_assert(SLOT_BYTES % 16 == 0 && SLOT_K % 16 == 0 && SLOT_V % 16 == 0, "alignment");
+  static_assert(QBUF_OFF % 16 == 0 && QBUF_BYTES % 16 == 0 && BAR_OFF % 8 == 0, "alignment");
   static_assert(GK >= 16 && GK % 16 == 0 && GV >= 16 && GV % 16 == 0,
                 "groups must cover whole 16-element steps");
 };
@@ -208,68 +230,82 @@ __device__ __forceinline__ void lds_param_pair(const uint32_t* p, uint32_t (&w0)
   }
 }
 
+// One span of a CTA's work: positions [t0, t1) of (batch row b, kv head hk,
+// head group hg); app_pos: first position the fused append writes (-1:
+// none); the result is the rows' final output (direct) or the partial result
+// at index ws_index of the rows' partial slots.
+struct Span {
+  int b, hk, hg, t0, t1, app_pos, ws_index;
+  bool direct;
+};
+
+// Bulk copy of span s's query rows (heads head0 .. head0 + nh - 1 of row
+// b, [head][D] in the query type) into a query buffer; thread 0 only.  The
+// rows are contiguous, start on a multiple of 128 bytes from the query base
+// (16-byte aligned, as the API requires) and are whole 16-byte units.
+template <class C>
+__device__ __forceinline__ void issue_q_rows(const DecodeArgs& a, const Span& s, uint8_t* dst,
+                                             uint64_t* bar) {
+  const int head0 = s.hk * a.gq + s.hg * a.heads_per_cta;
+  const int nh = min(a.heads_per_cta, a.gq - s.hg * a.heads_per_cta);
+  const int es = a.q_dtype == KVQ_F32 ? 4 : 2;
+  const uint32_t bytes = static_cast<uint32_t>(nh * C::D * es);
+  mbar_arrive_expect_tx(bar, bytes);
+  bulk_copy_g2s(dst,
+                static_cast<const uint8_t*>(a.q) +
+                    (static_cast<size_t>(s.b) * a.q_heads + head0) * C::D * es,
+                bytes, bar);
+}
+
 // FUSED: the instance used by the fused append + decode call (the append
 // prologue is compiled only there, so the plain decode keeps its registers
 // and schedule).
-template <class C, bool FUSED>
-__global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a) {
+// One span cur: the copy pipeline, the online softmax and the four warps'
+// merge.  Each warp's copies form one stream over the CTA's spans: stage g of
+// the stream lands in slot g mod kSlots with phase parity (g / kSlots) mod 2.
+// g0: stages of this warp's stream before cur (advanced by cur's stages);
+// pre: cur's stages already issued by the previous span (replaced by the
+// next span's; meaningful in lane 0, which issues).  peek(s) gives the CTA's
+// next span (false: none) and next(s) moves on to it.  The next span's
+// query rows go out at cur's start (query buffer (qspan + 1) mod 2; cur's
+// are in buffer qspan mod 2; qspan: the CTA's spans so far, kept in shared
+// memory), and the slots that cur's last stages free are
+// refilled with its first stages (not in the fused instance, whose append
+// comes first, nor with the paged layout, whose page lookups would stall
+// the warp), so that the next span starts without waiting (rotated keys
+// transform their own copy of the rows instead).
+// Returns true when a wait ran out (the CTA then stops; the rows are
+// flagged).
+template <class C, bool FUSED, class PeekFn, class NextFn>
+__device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, const Span& cur,
+                                            PeekFn&& peek, NextFn&& next, Span& nxt,
+                                            bool& has_next, int ws_stride, int& g0, int& pre) {
   constexpr int D = C::D, NGK = C::NGK, NGV = C::NGV, NQ = C::NQ, NP = C::NP, QS = C::QS;
   constexpr int HT = C::HT, KSTEPS = C::KSTEPS, GK = C::GK, GV = C::GV;
-  extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* wbuf = reinterpret_cast<uint16_t*>(smem + C::RING_BYTES);  // staged weights
-  float* alph = reinterpret_cast<float*>(smem + C::RING_BYTES + C::WB_BYTES);  // [warp][8]
-  float* mrg = alph + C::ALPHA_FLOATS;                                     // merge area
-  uint64_t* full = reinterpret_cast<uint64_t*>(mrg + C::MERGE_FLOATS);    // [warp][slot]
-
-  const int split = blockIdx.x;
-  const int hk = blockIdx.y / a.head_groups;
-  const int hg = blockIdx.y % a.head_groups;
-  const int b = blockIdx.z;
+  float* alph = reinterpret_cast<float*>(smem + C::ALPHA_OFF);          // [warp][8]
+  float* mrg = alph + C::ALPHA_FLOATS;                                  // merge area
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);      // [warp][slot]
+  uint64_t* qfull = full + C::kWarps * C::kSlots;                       // [query buffer]
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   uint64_t* wfull = full + warp * C::kSlots;
-  if (lane == 0) {
-    for (int sl = 0; sl < C::kSlots; ++sl) mbar_init(&wfull[sl], 1);
-    fence_barrier_init();
-  }
-  pdl_wait();
-  pdl_trigger();
-
-  int len = a.seq_lens[b];
-  const int lim = min(a.max_seq_len, a.capacity);
-  // fused append: positions [len - n_new, len) are written first; a row
-  // whose length is out of range appends nothing
-  int app_pos = -1;
-  if (FUSED && a.k_new != nullptr && len <= lim) {
-    if (len < a.n_new) {
-      if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0) flag_error(a.err, KVQ_DEVERR_BAD_POS);
-    } else {
-      app_pos = len - a.n_new;
-    }
-  }
-  if (len < 0 || len > lim) {
-    if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0) flag_error(a.err, KVQ_DEVERR_SEQ_LEN);
-    len = max(0, min(len, lim));
-  }
-  const int t0 = split * a.split_tokens;
+  const int b = cur.b, hk = cur.hk, hg = cur.hg, t0 = cur.t0, t1 = cur.t1;
+  const int app_pos = cur.app_pos, ws_index = cur.ws_index;
+  const bool direct = cur.direct;
   const int head0 = hk * a.gq + hg * a.heads_per_cta;
   const int nh = min(a.heads_per_cta, a.gq - hg * a.heads_per_cta);
-  if (t0 >= len) {
-    // an empty sequence attends to nothing: its output rows are zero
-    if (a.direct && len == 0 && split == 0)
-      for (int i = threadIdx.x; i < nh * D; i += C::kThreads)
-        store_out(a.out, a.out_dtype,
-                  (static_cast<size_t>(b) * a.q_heads + head0 + i / D) * D + i % D, 0.0f);
-    return;
-  }
-  const int t1 = min(t0 + a.split_tokens, len);
   const int n_tok = t1 - t0;
   const size_t slot = static_cast<size_t>(b) * a.kv_heads + hk;
 
   // ---- this warp's copy pipeline: positions [it*kStageTokens + 16*TPW*warp, +16*TPW)
-  // of the split for it = 0 .. my_iters-1, kSlots copies in flight.
+  // of a span for it = 0 .. iters-1, kSlots copies in flight.
   const int my_first = warp * 16 * C::TPW;
-  const int my_iters = n_tok > my_first ? (n_tok - my_first + C::kStageTokens - 1) / C::kStageTokens : 0;
+  auto iters_of = [&](const Span& s) {
+    const int n = s.t1 - s.t0;
+    return n > my_first ? (n - my_first + C::kStageTokens - 1) / C::kStageTokens : 0;
+  };
+  const int my_iters = iters_of(cur);
   uint8_t* wring = smem + warp * C::kSlots * C::SLOT_BYTES;
   // A stage's 16*TPW positions start at a multiple of 16*TPW, so they never
   // span two pages of the paged layout (pages hold a power of two >= 32).
@@ -278,16 +314,16 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
   // slot * capacity + tb of the per-position arrays.  Paged layout: its page
   // (block-table entry, looked up ahead by page_of) and the row inside
   // (page, kv head); a page outside the pool is never read.
-  auto page_of = [&](int it) -> int {
-    const int tb = t0 + it * C::kStageTokens + my_first;
-    return a.block_table[static_cast<size_t>(b) * a.pages_per_seq + (tb >> a.page_shift)];
+  auto page_of = [&](const Span& s, int it) -> int {
+    const int tb = s.t0 + it * C::kStageTokens + my_first;
+    return a.block_table[static_cast<size_t>(s.b) * a.pages_per_seq + (tb >> a.page_shift)];
   };
-  auto issue = [&](int it, int sl, int page) {
+  auto issue = [&](const Span& s, int it, int sl, int page) {
     const int base = it * C::kStageTokens + my_first;  // multiple of 16
-    const int n16 = (min(16 * C::TPW, n_tok - base) + 15) & ~15;
-    const int tb = t0 + base;
+    const int n16 = (min(16 * C::TPW, s.t1 - s.t0 - base) + 15) & ~15;
+    const int tb = s.t0 + base;
     uint8_t* dst = wring + sl * C::SLOT_BYTES;
-    size_t r = slot * a.capacity + tb;
+    size_t r = (static_cast<size_t>(s.b) * a.kv_heads + s.hk) * a.capacity + tb;
     if (a.block_table != nullptr) {
       if (page < 0 || page >= a.num_pages) {
         // no page: nothing is read (the row's output is unspecified); the
@@ -297,7 +333,7 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         return;
       }
       const int local = tb & ((1 << a.page_shift) - 1);
-      r = ((static_cast<size_t>(page) * a.kv_heads + hk) << a.page_shift) + local;
+      r = ((static_cast<size_t>(page) * a.kv_heads + s.hk) << a.page_shift) + local;
     }
     const uint32_t kbytes = n16 * C::KROW, vbytes = (n16 / 16) * C::VTILE;
     const uint32_t pkbytes = n16 * C::PROWK, pvbytes = n16 * C::PROWV;
@@ -314,17 +350,53 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
                   reinterpret_cast<const uint8_t*>(a.v_params) + r * C::PROWV, pvbytes,
                   &wfull[sl]);
   };
-  // First stages.  With a fused append, the stages that end before the new
-  // positions go out first, so that their copies overlap the append.
-  int first_pending = min(C::kSlots, my_iters);
-  if (lane == 0)
-    for (int it = 0; it < min(C::kSlots, my_iters); ++it) {
-      if (FUSED && app_pos >= 0 && t0 + it * C::kStageTokens + my_first + 16 * C::TPW > app_pos) {
-        first_pending = it;
-        break;
-      }
-      issue(it, it, a.block_table != nullptr ? page_of(it) : 0);
+  int issued = pre;  // stages of the stream from g0 on that are in flight or consumed
+  // the next span's query rows
+  const bool q_bulk = !a.rotate_q;
+  uint8_t* qbuf = smem + C::QBUF_OFF;
+  // ctl[0]: spans begun before cur; ctl[1]: the next span's rows are in
+  // flight; ctl[2]: a query wait ran out (the CTA stops after this span)
+  int* ctl = reinterpret_cast<int*>(smem + C::CTL_OFF);
+  if (q_bulk && threadIdx.x == 0) {
+    Span s;
+    const int qs = ctl[0];
+    ctl[1] = 0;
+    if (peek(s)) {
+      issue_q_rows<C>(a, s, qbuf + ((qs + 1) & 1) * C::QBUF_BYTES, &qfull[(qs + 1) & 1]);
+      ctl[1] = 1;
     }
+  }
+  // this warp's view of the next span for the refills at cur's end (b, hk,
+  // t0, t1; b < 0: none), kept in shared memory rather than registers (read
+  // through a volatile pointer, so that the reads stay where they are used)
+  volatile int* wnext = ctl + 4 + 4 * warp;
+  if (!FUSED && a.block_table == nullptr && lane == 0) {
+    Span s;
+    const bool any = peek(s);
+    wnext[0] = any ? s.b : -1;
+    wnext[1] = s.hk;
+    wnext[2] = s.t0;
+    wnext[3] = s.t1;
+  }
+  // First stages (those the previous span has not issued).  With a fused
+  // append, the stages that end before the new positions go out first, so
+  // that their copies overlap the append.
+  int first_pending = min(C::kSlots, my_iters);
+  if (lane == 0) {
+    if constexpr (FUSED) {
+      for (int it = 0; it < min(C::kSlots, my_iters); ++it) {
+        if (app_pos >= 0 && t0 + it * C::kStageTokens + my_first + 16 * C::TPW > app_pos) {
+          first_pending = it;
+          break;
+        }
+        issue(cur, it, (g0 + it) % C::kSlots, a.block_table != nullptr ? page_of(cur, it) : 0);
+      }
+    } else {
+      for (; issued < min(C::kSlots, my_iters); ++issued)
+        issue(cur, issued, (g0 + issued) % C::kSlots,
+              a.block_table != nullptr ? page_of(cur, issued) : 0);
+    }
+  }
   if constexpr (FUSED) {
     // ---- fused append of the new positions in this split (every head-group
     // CTA of the slot writes the same bytes), made visible to the bulk
@@ -350,12 +422,15 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     }
     if (lane == 0)
       for (int it = first_pending; it < min(C::kSlots, my_iters); ++it)
-        issue(it, it, a.block_table != nullptr ? page_of(it) : 0);
+        issue(cur, it, (g0 + it) % C::kSlots, a.block_table != nullptr ? page_of(cur, it) : 0);
+    issued = min(C::kSlots, my_iters);
   }
   __syncwarp();
 
   // ------------------------------------------------------------ consumers
   const int g = lane >> 2, c = lane & 3;
+  bool timed_out = false;
+  int consumed = 0;  // stages of cur this warp has consumed
   float m_run[HT], l_run[HT];
   float oacc[KSTEPS][NP][4];
   float2 zacc[HT][NGV];  // zero term, score layout: (row g, row g+8) partials
@@ -404,37 +479,53 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       }
       qrot = qs;
     }
+    // the query buffer, or the rotated rows
+    const int qs = ctl[0];
+    uint8_t* qcur = qbuf + (qs & 1) * C::QBUF_BYTES;
+    if (q_bulk) {
+      // (a wait that runs out is flagged, noted in ctl[2], and stops the
+      // CTA at the span's end; the span runs on meanwhile)
+      if (!mbar_wait_bounded(&qfull[qs & 1], (qs >> 1) & 1, a.err, a.wait_limit_ns))
+        ctl[2] = 1;
+    }
     float qraw[NQ][KSTEPS][4];
     float amax = 0.0f;
 #pragma unroll
     for (int nt = 0; nt < NQ; ++nt) {
       const int n = 8 * nt + g;
       const int head = QS == 2 ? n / 2 : n;
-      const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * D;
 #pragma unroll
       for (int j = 0; j < KSTEPS; ++j)
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          // elements d, d+1 with d = 16j + 2c + 8r
-          const size_t d = row + 16 * j + 2 * c + 8 * r;
-          float2 v = make_float2(0.0f, 0.0f);
-          if (head < nh && qrot != nullptr) {
+          float2 v;
+          if (qrot != nullptr) {
+            // elements d, d+1 with d = 16j + 2c + 8r
             constexpr float kInvD = 1.0f / D;  // exact: D is a power of two
             const float* x = qrot + head * D + 16 * j + 2 * c + 8 * r;
-            v = make_float2(x[0] * kInvD, x[1] * kInvD);
-          } else if (head < nh) {
+            const bool in = head < nh;
+            v = in ? make_float2(x[0] * kInvD, x[1] * kInvD) : make_float2(0.0f, 0.0f);
+          } else {
+            // elements d, d+1 with d = 16j + 2c + 8r of this head's row
+            const int d = head * D + 16 * j + 2 * c + 8 * r;
+            const bool in = head < nh;
+            uint32_t u = 0u, u1 = 0u;
             if (a.q_dtype == KVQ_F32) {
-              v = __ldg(reinterpret_cast<const float2*>(a.q) + d / 2);
+              const uint2 w = in ? *reinterpret_cast<const uint2*>(qcur + 4 * d) : make_uint2(0u, 0u);
+              u = w.x;
+              u1 = w.y;
             } else {
-              const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(a.q) + d / 2);
-              v = a.q_dtype == KVQ_BF16
-                      ? make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u))
-                      : unpack_half2(u);
+              u = in ? *reinterpret_cast<const uint32_t*>(qcur + 2 * d) : 0u;
             }
+            v = a.q_dtype == KVQ_F32
+                    ? make_float2(__uint_as_float(u), __uint_as_float(u1))
+                : a.q_dtype == KVQ_BF16
+                    ? make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u))
+                    : unpack_half2(u);
           }
           qraw[nt][j][2 * r] = v.x;
           qraw[nt][j][2 * r + 1] = v.y;
-          amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
+          amax = fmaxf(amax, fmaxf(fabsf(qraw[nt][j][2 * r]), fabsf(qraw[nt][j][2 * r + 1])));
         }
     }
     if (qrot != nullptr) __syncthreads();  // every warp has read qs before any stages weights
@@ -790,16 +881,16 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       __syncwarp();
     };
 
-    int sl = 0;
-    uint32_t phase = 0;
+    int sl = g0 % C::kSlots;
+    uint32_t phase = (g0 / C::kSlots) & 1;
     int it = 0;
     for (; it < my_iters; ++it) {
-      // paged layout: the page of the stage this slot is refilled with,
-      // looked up before the arithmetic so that the block-table read
-      // overlaps it
+      // the stage this slot is refilled with (this span's or, past its end,
+      // the next span's); paged layout: its page, looked up before the
+      // arithmetic so that the block-table read overlaps it
+      const bool refill = it + C::kSlots < my_iters;
       int next_page = 0;
-      if (a.block_table != nullptr && lane == 0 && it + C::kSlots < my_iters)
-        next_page = page_of(it + C::kSlots);
+      if (a.block_table != nullptr && lane == 0 && refill) next_page = page_of(cur, it + C::kSlots);
       if (!mbar_wait_bounded(&wfull[sl], phase, err, a.wait_limit_ns)) break;
       const uint8_t* st = wring + sl * C::SLOT_BYTES;
       const int base = it * C::kStageTokens + my_first;  // first position of this slot
@@ -816,30 +907,60 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
         }
       }
       __syncwarp();
-      if (lane == 0 && it + C::kSlots < my_iters) {
-        // the warp's reads of this slot are done (registers); hand it back to
-        // the copy engine for a later stage
-        fence_proxy_async_shared();
-        issue(it + C::kSlots, sl, next_page);
+      if (lane == 0) {
+        // the warp's reads of this slot are done (registers); hand it back
+        // to the copy engine for a later stage: cur's, or past its end the
+        // next span's (in order: stage `issued` of the stream)
+        if (refill) {
+          fence_proxy_async_shared();
+          issue(cur, it + C::kSlots, sl, next_page);
+          ++issued;
+        } else if (!FUSED && a.block_table == nullptr && it + C::kSlots == issued &&
+                   wnext[0] >= 0) {
+          Span s;
+          s.b = wnext[0];
+          s.hk = wnext[1];
+          s.t0 = wnext[2];
+          s.t1 = wnext[3];
+          if (issued - my_iters < iters_of(s)) {
+            fence_proxy_async_shared();
+            issue(s, issued - my_iters, sl, 0);
+            ++issued;
+          }
+        }
       }
       if (++sl == C::kSlots) {
         sl = 0;
         phase ^= 1u;
       }
     }
-    // Drain (only after a timed-out wait): copies issued but not consumed
-    // must land before shared memory is reused; bounded in any case.
-    if (it < my_iters && lane == 0) {
-      for (int k = it; k < min(my_iters, it + C::kSlots); ++k)
-        mbar_wait_bounded(&wfull[k % C::kSlots], (k / C::kSlots) & 1, err, a.wait_limit_ns);
-    }
+    timed_out = it < my_iters;
+    consumed = it;
+  }
+  // the next span: its first stages and its query elements are requested
+  // before the merge, so that they arrive during it (the elements always,
+  // so that their registers are free during the main loop; without a next
+  // span they are cur's again, unused)
+  has_next = next(nxt);
+  if (!FUSED && has_next && !timed_out && lane == 0) {
+    const int n = min(C::kSlots, iters_of(nxt));
+    for (; issued < my_iters + n; ++issued)
+      issue(nxt, issued - my_iters, (g0 + issued) % C::kSlots,
+            a.block_table != nullptr ? page_of(nxt, issued - my_iters) : 0);
   }
 
   // ------------------------------------------------------------ epilogue
-  // with one split per row this CTA's result is final
-  const bool direct = a.direct;
-  __syncthreads();  // all stages consumed; the ring becomes the merge buffer
-  float* ob = reinterpret_cast<float*>(smem);  // [warp][8][D]
+  // all stages consumed; a wait that ran out stops the CTA, after the copies
+  // still in flight (this span's and the next one's) have landed: shared
+  // memory must not be left to them; bounded in any case
+  const bool aborted = __syncthreads_or(timed_out || ctl[2] != 0);
+  // (query rows still in flight are waited for at the kernel's end)
+  if (aborted && lane == 0)
+    for (int k = g0 + consumed; k < g0 + issued; ++k)
+      mbar_wait_bounded(&wfull[k % C::kSlots], (k / C::kSlots) & 1, a.err, a.wait_limit_ns);
+  g0 += my_iters;
+  pre = issued - my_iters;
+  float* ob = reinterpret_cast<float*>(wbuf);  // [warp][OB_HEADS][D]
   float* mb = mrg;                             // [warp][8]
   float* lb = mb + C::kWarps * 8;              // [warp][8]
   float* zb = lb + C::kWarps * 8;              // [warp][8][NGV]
@@ -875,8 +996,8 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
       for (int j = 0; j < KSTEPS; ++j) {
         const float s0 = pow2i(24 - u_run - field_pos<C::BV>((2 * j) % (16 / C::BV)));
         const float s1 = pow2i(24 - u_run - field_pos<C::BV>((2 * j + 1) % (16 / C::BV)));
-        ob[(warp * 8 + head) * D + 16 * j + g] = (oacc[j][pt][0] + oacc[j][pt][1]) * s0;
-        ob[(warp * 8 + head) * D + 16 * j + 8 + g] = (oacc[j][pt][2] + oacc[j][pt][3]) * s1;
+        ob[(warp * C::OB_HEADS + head) * D + 16 * j + g] = (oacc[j][pt][0] + oacc[j][pt][1]) * s0;
+        ob[(warp * C::OB_HEADS + head) * D + 16 * j + 8 + g] = (oacc[j][pt][2] + oacc[j][pt][3]) * s1;
       }
     }
   }
@@ -896,24 +1017,204 @@ __global__ void __launch_bounds__(C::kThreads) decode_kernel(const DecodeArgs a)
     }
     rden[head] = __frcp_rn(den);
     if (!direct) {
-      const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * a.num_splits + split;
+      const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * ws_stride + ws_index;
       a.ws_lse[row] = M + __log2f(den);
     }
   }
+  if (threadIdx.x == 0) ++ctl[0];  // every thread read it in the prologue
   __syncthreads();
   for (int idx = threadIdx.x; idx < nh * D; idx += C::kThreads) {
     const int head = idx / D, d = idx % D;
     float num = 0.0f;
 #pragma unroll
     for (int w = 0; w < C::kWarps; ++w)
-      num = fmaf(wt[head * C::kWarps + w], ob[(w * 8 + head) * D + d] + zb[(w * 8 + head) * NGV + d / GV], num);
+      num = fmaf(wt[head * C::kWarps + w], ob[(w * C::OB_HEADS + head) * D + d] + zb[(w * 8 + head) * NGV + d / GV], num);
     if (direct) {
       store_out(a.out, a.out_dtype, (static_cast<size_t>(b) * a.q_heads + head0 + head) * D + d,
                 num * rden[head]);
     } else {
-      const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * a.num_splits + split;
+      const size_t row = (static_cast<size_t>(b) * a.q_heads + head0 + head) * ws_stride + ws_index;
       a.ws_o[row * D + d] = num * rden[head];
     }
+  }
+  return aborted;
+}
+
+// The decode kernel: one span per CTA on the per-row split grid (grid =
+// (splits, kv heads x head groups, batch rows)), or, with stream_q > 0, the
+// balanced (stream-K) schedule: the positions of every
+// (batch row, kv head, head group) unit are cut into stages of kStageTokens;
+// the units' stages, row after row, form one sequence of S stages, and CTA c
+// of the one-wave grid takes stages [c*Q, (c+1)*Q), Q = max(stream_q,
+// ceil(S / grid)), so that every CTA streams the same number of stages
+// whatever the row lengths.  A unit that one CTA covers whole is written
+// directly; the others leave one partial result per covering CTA (index:
+// the CTA's rank among them) for the combine kernel.  The balanced schedule
+// takes at most kStreamRows rows.
+template <class C, bool FUSED>
+__global__ void __launch_bounds__(C::kThreads, FUSED ? C::kMinBlocks - 1 : C::kMinBlocks)
+    decode_kernel(const DecodeArgs a) {
+  constexpr int D = C::D, T = C::kStageTokens;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);  // [warp][slot]
+  uint64_t* qfull = full + C::kWarps * C::kSlots;                   // [query buffer]
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint64_t* wfull = full + warp * C::kSlots;
+  if (lane == 0) {
+    for (int sl = 0; sl < C::kSlots; ++sl) mbar_init(&wfull[sl], 1);
+    if (warp == 0) {
+      mbar_init(&qfull[0], 1);
+      mbar_init(&qfull[1], 1);
+      reinterpret_cast<int*>(smem + C::CTL_OFF)[0] = 0;  // spans begun
+      reinterpret_cast<int*>(smem + C::CTL_OFF)[1] = 0;  // next span's query rows in flight
+      reinterpret_cast<int*>(smem + C::CTL_OFF)[2] = 0;  // a query wait ran out
+    }
+    fence_barrier_init();
+  }
+  const int lim = min(a.max_seq_len, a.capacity);
+  const bool stream = a.stream_q > 0;
+
+  // balanced schedule: the rows' lengths and the prefix sums of their stages,
+  // built before the wait for the previous grid (no kernel of this library
+  // writes the lengths; the ring is free scratch until the first span)
+  int* lens = reinterpret_cast<int*>(smem + C::SMEM_BYTES - 4 * (2 * kStreamRows + 1));
+  int* off = lens + kStreamRows;
+  const int U = a.kv_heads * a.head_groups;
+  int p = 0, p_end = 0, Q = 1, rb = 0;
+  if (stream) {
+    stream_row_offsets(a.seq_lens, a.batch, lim, U, T, off, lens, reinterpret_cast<int*>(smem));
+    const int S = off[kStreamRows];  // rows past the batch count no stages
+    Q = max(a.stream_q, (S + gridDim.x - 1) / gridDim.x);
+    p = blockIdx.x * Q;
+    p_end = min(p + Q, S);
+    // the row holding stage p (rows with no stages are skipped)
+    while (rb < a.batch - 1 && off[rb + 1] <= p) ++rb;
+  }
+  pdl_wait();
+  pdl_trigger();
+  if (stream && blockIdx.x == 0)
+    for (int r = threadIdx.x; r < a.batch; r += C::kThreads)
+      if (lens[r] < 0 || lens[r] > lim) flag_error(a.err, KVQ_DEVERR_SEQ_LEN);
+
+  // Span of the balanced schedule at stage p of row rb: stages [j0, j1) of
+  // unit u; adv = j1 - j0.
+  auto stream_span = [&](int pp, int r, Span& s, int& adv) {
+    const int ns = (off[r + 1] - off[r]) / U;  // stages of each unit of row r
+    const int q0 = pp - off[r];
+    const int u = q0 / ns;
+    const int j0 = q0 % ns;
+    const int j1 = min(ns, j0 + (p_end - pp));
+    s.b = r;
+    s.hk = u / a.head_groups;
+    s.hg = u % a.head_groups;
+    s.t0 = j0 * T;
+    const int len_raw = lens[r];
+    s.t1 = min(max(0, min(len_raw, lim)), j1 * T);
+    // fused append: as on the split grid; a row shorter than the new rows
+    // is flagged once (by the CTA holding its first unit's first stage)
+    s.app_pos = -1;
+    if (FUSED && a.k_new != nullptr && len_raw <= lim) {
+      if (len_raw >= a.n_new)
+        s.app_pos = len_raw - a.n_new;
+      else if (u == 0 && j0 == 0 && threadIdx.x == 0)
+        flag_error(a.err, KVQ_DEVERR_BAD_POS);
+    }
+    const int ubase = off[r] + u * ns;  // the unit's first stage
+    s.ws_index = blockIdx.x - ubase / Q;
+    s.direct = ubase / Q == (ubase + ns - 1) / Q;
+    adv = j1 - j0;
+  };
+
+  Span cur;
+  int adv = 0;
+  // the first span's query rows are requested first (query buffer 0)
+  const bool q_bulk = !a.rotate_q;
+  auto first_q = [&]() {
+    if (q_bulk && threadIdx.x == 0) issue_q_rows<C>(a, cur, smem + C::QBUF_OFF, &qfull[0]);
+  };
+  if (stream) {
+    if (p >= p_end) return;
+    stream_span(p, rb, cur, adv);
+    first_q();
+  } else {
+    const int split = blockIdx.x;
+    cur.hk = blockIdx.y / a.head_groups;
+    cur.hg = blockIdx.y % a.head_groups;
+    cur.b = blockIdx.z;
+    int len = a.seq_lens[cur.b];
+    // fused append: positions [len - n_new, len) are written first; a row
+    // whose length is out of range appends nothing
+    cur.app_pos = -1;
+    if (FUSED && a.k_new != nullptr && len <= lim) {
+      if (len < a.n_new) {
+        if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+          flag_error(a.err, KVQ_DEVERR_BAD_POS);
+      } else {
+        cur.app_pos = len - a.n_new;
+      }
+    }
+    if (len < 0 || len > lim) {
+      if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+        flag_error(a.err, KVQ_DEVERR_SEQ_LEN);
+      len = max(0, min(len, lim));
+    }
+    cur.t0 = split * a.split_tokens;
+    if (cur.t0 >= len) {
+      // an empty sequence attends to nothing: its output rows are zero
+      const int head0 = cur.hk * a.gq + cur.hg * a.heads_per_cta;
+      const int nh = min(a.heads_per_cta, a.gq - cur.hg * a.heads_per_cta);
+      if (a.direct && len == 0 && split == 0)
+        for (int i = threadIdx.x; i < nh * D; i += C::kThreads)
+          store_out(a.out, a.out_dtype,
+                    (static_cast<size_t>(cur.b) * a.q_heads + head0 + i / D) * D + i % D, 0.0f);
+      return;
+    }
+    cur.t1 = min(cur.t0 + a.split_tokens, len);
+    cur.ws_index = split;
+    cur.direct = a.direct;
+    first_q();
+  }
+
+  int g0 = 0, pre = 0;  // this warp's copy stream (see decode_span)
+  // the CTA's span after the one at stage p (split grid: none): peek only
+  // looks, next moves on
+  auto peek = [&](Span& s) {
+    if (!stream) return false;
+    const int pp = p + adv;
+    if (pp >= p_end) return false;
+    int r = rb;
+    while (r < a.batch - 1 && off[r + 1] <= pp) ++r;
+    int ad;
+    stream_span(pp, r, s, ad);
+    return true;
+  };
+  auto next = [&](Span& s) {
+    if (!stream) return false;
+    p += adv;
+    while (rb < a.batch - 1 && off[rb + 1] <= p) ++rb;
+    if (p >= p_end) return false;
+    stream_span(p, rb, s, adv);
+    return true;
+  };
+  for (bool first = true;; first = false) {
+    // the previous span's merge is done with shared memory before this
+    // span's prologue and first tile reuse it
+    if (!first) __syncthreads();
+    Span nxt = cur;
+    bool has_next = false;
+    if (decode_span<C, FUSED>(a, smem, cur, peek, next, nxt, has_next, a.num_splits, g0, pre) ||
+        !has_next)
+      break;
+    cur = nxt;
+  }
+  // after a wait ran out: query rows still in flight land before the CTA
+  // ends (the last span's, if its wait ran out, and the next span's)
+  const int* ctl = reinterpret_cast<const int*>(smem + C::CTL_OFF);
+  if (threadIdx.x == 0 && (ctl[1] != 0 || ctl[2] != 0)) {
+    const int last = ctl[0] - 1;
+    if (ctl[2]) mbar_wait_bounded(&qfull[last & 1], (last >> 1) & 1, a.err, a.wait_limit_ns);
+    if (ctl[1]) mbar_wait_bounded(&qfull[(last + 1) & 1], ((last + 1) >> 1) & 1, a.err, a.wait_limit_ns);
   }
 }
 
@@ -933,6 +1234,7 @@ DecodeKernel make_decode_kernel() {
   k.launch_fused = &launch_decode<C, true>;
   k.tile = 64;
   k.max_per_sm = 0;
+  k.stage_tokens = C::kStageTokens;
   return k;
 }
 

@@ -796,6 +796,7 @@ DecodeKernel make_decode_tc_kernel() {
   k.launch_fused = nullptr;
   k.tile = C::TILE;
   k.max_per_sm = 1;  // all 512 tensor-memory columns of the SM
+  k.stage_tokens = 0;
   return k;
 }
 

@@ -8,6 +8,10 @@
 
 namespace kvq {
 
+// Rows a balanced (stream-K) decode schedules at most (their prefix sums
+// live in shared memory).
+constexpr int kStreamRows = 256;
+
 // Launches `kernel` with programmatic stream serialization: its blocks may
 // start while the previous kernel in the stream finishes, and wait for it in
 // pdl_wait() before touching global memory.  Captured into CUDA graphs as a
@@ -65,7 +69,10 @@ struct DecodeArgs {
   int heads_per_cta;  // <= 8
   int head_groups;    // ceil(gq / heads_per_cta)
   int split_tokens;   // multiple of 64
-  int num_splits;     // grid.x
+  int num_splits;     // grid.x; balanced schedule: partial slots per row
+  // Balanced (stream-K) schedule when > 0: grid.x CTAs share the rows' stages
+  // evenly, at least stream_q stages each (plain decode only).
+  int stream_q;
   float sm_scale_log2;  // softmax scale times log2(e)
   bool rotate_q;        // keys are stored rotated: use H q / D
   const int32_t* block_table;  // paged layout, as in QuantizeArgs (NULL: slots)
@@ -102,6 +109,7 @@ struct DecodeKernel {
   int smem_bytes;
   int tile;              // split lengths are rounded to a multiple of this
   int max_per_sm;        // CTAs per SM the kernel allows itself (0: no limit of its own)
+  int stage_tokens;      // positions per stage of the balanced schedule (0: not supported)
   cudaError_t (*launch)(const DecodeArgs&, dim3 grid, cudaStream_t stream);
   cudaError_t (*launch_fused)(const DecodeArgs&, dim3 grid, cudaStream_t stream);
 };
@@ -122,6 +130,9 @@ struct CombineArgs {
   void* out;
   int out_dtype;
   int batch, q_heads, head_dim, capacity, max_seq_len, split_tokens, num_splits;
+  // balanced schedule of the decode (stream_q > 0): its grid size, stage
+  // length and unit layout, from which each row's count of partials follows
+  int stream_q, stream_grid, stage_tokens, kv_heads, head_groups, gq, heads_per_cta;
 };
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);

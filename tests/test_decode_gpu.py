@@ -161,3 +161,29 @@ def test_single_split_needs_no_workspace():
     out = kvq.kvq_decode_attention(cache, q, lens, 64)  # no workspace
     torch.cuda.synchronize()
     assert torch.isfinite(out).all()
+
+
+@pytest.mark.parametrize("lens", [[1000, 613, 77, 0, 2048, 129], [4096], [300, 0, 0, 5000]])
+def test_balanced_schedule(ora, lens, monkeypatch):
+    # the opt-in one-wave schedule: spans cross unit and row boundaries
+    monkeypatch.setenv("KVQ_DECODE_SCHEDULE", "balanced")
+    out, ref = _run(ora, len(lens), 2, 8, 128, 4, 2, 64, lens, seed=21 + len(lens))
+    compare_attention(out, ref)
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert not out[b].any()
+
+
+@pytest.mark.parametrize("q_dtype,offset", [(torch.bfloat16, 1), (torch.float32, 1),
+                                            (torch.float16, 4)])
+def test_unaligned_query_is_rejected(q_dtype, offset):
+    # the query rows are bulk-copied: a query not on 16 bytes is an invalid
+    # argument, and nothing is launched
+    cache = kvq.KVCache.allocate(1, 1, 128, 64, 4, 2, 64)
+    buf = torch.zeros(4 * 128 + offset, dtype=q_dtype, device="cuda")
+    q = buf[offset:].view(1, 4, 128)
+    assert q.data_ptr() % 16 != 0
+    lens = torch.tensor([64], dtype=torch.int32, device="cuda")
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_decode_attention(cache, q, lens, 64)
+    assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
