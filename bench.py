@@ -51,8 +51,11 @@ METRIC = "quantized-KV decode attention HBM GB/s (% of B200 peak) and KV-tokens/
 FALLBACK_HBM_GBS = 6650.0
 DEFAULT_WORKLOAD = "ragged"
 # every (workload, bits) configuration, recorded in the "configs" key
-CONFIG_SWEEP = (("tiny", (4, 2)), ("llama3_8b", (4, 2)), ("long", (8, 4)), ("long", (4, 2)),
-                ("ragged", (4, 2)), ("qwen_mistral", (4, 2)), ("qwen_mistral", (2, 4)))
+# (workload, bits, append fused into the decode call)
+CONFIG_SWEEP = (("tiny", (4, 2), False), ("llama3_8b", (4, 2), False), ("long", (8, 4), False),
+                ("long", (8, 4), True), ("long", (4, 2), False), ("ragged", (4, 2), False),
+                ("qwen_mistral", (4, 2), False), ("qwen_mistral", (4, 2), True),
+                ("qwen_mistral", (2, 4), False))
 KERNEL_REPS = 60  # isolated graph replays per kernel time (median)
 
 
@@ -341,10 +344,10 @@ def kernel_rooflines(arm, w, kern, nbytes, reps, rotate_keys=False):
     return roof
 
 
-def measure_config(name, bits, device, reps):
+def measure_config(name, bits, device, reps, fused=False):
     """Per-kernel device times and rooflines of one configuration's step."""
     w = workloads.WORKLOADS[name]
-    arm, rotate = make_arm(w, bits, device, 3)
+    arm, rotate = make_arm(w, bits, device, 3, fused=fused)
     for i in range(3):
         arm.step(i % rotate)
     torch.cuda.synchronize()
@@ -355,7 +358,8 @@ def measure_config(name, bits, device, reps):
     dec = roof["decode_attention"]
     entry = {
         "workload": name, "bits": f"K{bits[0]}V{bits[1]}",
-        "step": step_name(w, arm),
+        "step": step_name(w, arm), "fused_append": arm.fused,
+        "step_kernels_ms": round(sum(k["ms"] for k in roof.values()), 5),
         "split_tokens": arm.split_tokens, "num_splits": arm.num_splits,
         "rotating_sets": rotate,
         "kv_tokens": nbytes["tokens"],
@@ -485,8 +489,8 @@ def run_ours(args, rank, world, device):
     torch.cuda.empty_cache()
     if not args.no_configs:
         with ClockSampler(physical_index()) as cclocks:
-            result["configs"] = [measure_config(n, b, device, KERNEL_REPS)
-                                 for n, b in CONFIG_SWEEP]
+            result["configs"] = [measure_config(n, b, device, KERNEL_REPS, fused=f)
+                                 for n, b, f in CONFIG_SWEEP]
         result["clocks_configs"] = cclocks.summary()
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, bits, args.cpu_seconds)

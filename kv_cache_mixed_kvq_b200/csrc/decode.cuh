@@ -1052,7 +1052,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
 // the CTA's rank among them) for the combine kernel.  The balanced schedule
 // takes at most kStreamRows rows.
 template <class C, bool FUSED>
-__global__ void __launch_bounds__(C::kThreads, FUSED ? C::kMinBlocks - 1 : C::kMinBlocks)
+__global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     decode_kernel(const DecodeArgs a) {
   constexpr int D = C::D, T = C::kStageTokens;
   extern __shared__ __align__(128) uint8_t smem[];

@@ -128,7 +128,12 @@ def test_rotation_exceeds_twice_the_l2():
 
 def test_config_sweep_covers_every_workload_and_bit_pair():
     import bench
-    got = {(n, b) for n, b in bench.CONFIG_SWEEP}
+    got = {(n, b) for n, b, _ in bench.CONFIG_SWEEP}
     want = {(n, b) for n, w in bench.workloads.WORKLOADS.items() for b in w.bits}
     assert got == want
+    # the fused append is measured beside the two-call step of every workload
+    # that appends during decode
+    fused = {n for n, _, f in bench.CONFIG_SWEEP if f}
+    appending = {n for n, w in bench.workloads.WORKLOADS.items() if w.append > 0}
+    assert fused == appending
     assert bench.DEFAULT_WORKLOAD == "ragged" and bench.KERNEL_REPS >= 50
