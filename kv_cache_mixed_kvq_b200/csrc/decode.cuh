@@ -378,6 +378,18 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
     wnext[2] = s.t0;
     wnext[3] = s.t1;
   }
+  // The fused append's input rows are requested into L2 before anything
+  // else, so that the append's loads below find them there.
+  if (FUSED && app_pos >= 0 && threadIdx.x == 0) {
+    const int p0 = max(app_pos, t0);
+    if (p0 < t1) {
+      const int es = a.in_dtype == KVQ_F32 ? 4 : 2;
+      const size_t row0 = slot * a.n_new + (p0 - app_pos);
+      const uint32_t bytes = static_cast<uint32_t>((t1 - p0) * D * es);
+      bulk_prefetch_l2(static_cast<const uint8_t*>(a.k_new) + row0 * D * es, bytes);
+      bulk_prefetch_l2(static_cast<const uint8_t*>(a.v_new) + row0 * D * es, bytes);
+    }
+  }
   // First stages (those the previous span has not issued).  With a fused
   // append, the stages that end before the new positions go out first, so
   // that their copies overlap the append.
