@@ -29,18 +29,23 @@ def _inputs(B, Hkv, T, D, seed, dtype=torch.bfloat16):
 
 
 class _Split:
+    """Split override (tokens), or "balanced" for the opt-in one-wave schedule."""
+
     def __init__(self, n):
         self.n = n
 
     def __enter__(self):
-        self.old = os.environ.get("KVQ_SPLIT_TOKENS")
-        if self.n:
+        self.old = {k: os.environ.get(k) for k in ("KVQ_SPLIT_TOKENS", "KVQ_DECODE_SCHEDULE")}
+        if self.n == "balanced":
+            os.environ["KVQ_DECODE_SCHEDULE"] = "balanced"
+        elif self.n:
             os.environ["KVQ_SPLIT_TOKENS"] = str(self.n)
 
     def __exit__(self, *exc):
-        os.environ.pop("KVQ_SPLIT_TOKENS", None)
-        if self.old is not None:
-            os.environ["KVQ_SPLIT_TOKENS"] = self.old
+        for k, v in self.old.items():
+            os.environ.pop(k, None)
+            if v is not None:
+                os.environ[k] = v
 
 
 def _gpu_row(cache, b):
@@ -128,7 +133,7 @@ def _fused_case(ora, D=128, bk=4, bv=2, G=64, gv=0, gq=4, n_new=1, lens=(200, 70
 
 
 @pytest.mark.parametrize("n_new", [1, 5, 16, 37])
-@pytest.mark.parametrize("split", [None, 64])
+@pytest.mark.parametrize("split", [None, 64, "balanced"])
 @pytest.mark.parametrize("gq", [4, 16])
 def test_fused_matches_oracle(ora, n_new, split, gq):
     # lengths put new tokens across the 64-position split boundaries
@@ -184,7 +189,7 @@ def test_rows_that_append_nothing(ora):
     compare_attention(out, ref, TOL)
 
 
-@pytest.mark.parametrize("split", [None, 64])
+@pytest.mark.parametrize("split", [None, 64, "balanced"])
 def test_fused_equals_two_calls(ora, split):
     # the fused call writes the same bytes as the append kernel and returns
     # the same bits as the separate decode

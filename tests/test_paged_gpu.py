@@ -45,18 +45,23 @@ def _decode(cache, q, lens, T, out_dtype=torch.float32):
 
 
 class _Split:
+    """Split override (tokens), or "balanced" for the opt-in one-wave schedule."""
+
     def __init__(self, n):
         self.n = n
 
     def __enter__(self):
-        self.old = os.environ.get("KVQ_SPLIT_TOKENS")
-        if self.n:
+        self.old = {k: os.environ.get(k) for k in ("KVQ_SPLIT_TOKENS", "KVQ_DECODE_SCHEDULE")}
+        if self.n == "balanced":
+            os.environ["KVQ_DECODE_SCHEDULE"] = "balanced"
+        elif self.n:
             os.environ["KVQ_SPLIT_TOKENS"] = str(self.n)
 
     def __exit__(self, *exc):
-        os.environ.pop("KVQ_SPLIT_TOKENS", None)
-        if self.old is not None:
-            os.environ["KVQ_SPLIT_TOKENS"] = self.old
+        for k, v in self.old.items():
+            os.environ.pop(k, None)
+            if v is not None:
+                os.environ[k] = v
 
 
 @pytest.mark.parametrize("P", [32, 64, 256])
@@ -101,7 +106,7 @@ def test_paged_rotated_keys_and_value_groups(ora):
     compare_attention(_decode(cache, q, [200, 133], cap), ref, TOL)
 
 
-@pytest.mark.parametrize("split", [None, 64, 128, 448])
+@pytest.mark.parametrize("split", [None, 64, 128, 448, "balanced"])
 @pytest.mark.parametrize("P", [32, 128])
 @pytest.mark.parametrize("gq,q_dtype", [(4, torch.bfloat16), (8, torch.float32)])
 def test_paged_decode_matches_oracle(ora, split, P, gq, q_dtype):
