@@ -364,6 +364,17 @@ int kvq_decode_attention_static(const kvq_cache_desc* cache, const void* q,
 /*
  * Tokens per split that kvq_decode_attention() will use for these
  * arguments on the current device (0 if invalid).  Informational.
+ *
+ * Environment read when a decode plan is made (plans are cached per shape
+ * and per these settings; results stay within the attention tolerance
+ * under every setting):
+ *   KVQ_SPLIT_TOKENS=n       split size override, a multiple of 64 (tests);
+ *   KVQ_DECODE_SCHEDULE=balanced  one wave of CTAs sharing all rows' stages
+ *                            equally (stream-K); slower than the default
+ *                            per-row splits on B200, kept for comparison;
+ *   KVQ_DECODE_KERNEL=tcgen05     the tensor-memory (tcgen05) decode kernel
+ *                            for head_dim 128; slower than the default,
+ *                            kept for comparison.
  */
 int32_t kvq_decode_split_tokens(const kvq_cache_desc* cache,
                                 int32_t num_q_heads, int32_t max_seq_len);

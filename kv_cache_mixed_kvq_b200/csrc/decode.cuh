@@ -21,6 +21,8 @@
 //    fp32 accumulate) multiply raw codes; the per-group scale and zero are
 //    applied afterwards:  q.k^ = sum_g scale_g (q . c_g) + zero_g sum_{d in g} q_d
 //    and  o = sum_t (p_t scale_t) c_t + sum_t p_t zero_t;
+//  * the query rows of each span are bulk-copied into one of two shared
+//    buffers (the next span's while the current one runs);
 //  * the query (B operand of the score product) is scaled by a power of two
 //    and split into binary16 high and low parts in two columns (the low part
 //    is zero for 16-bit queries); the weights p_t * scale_t (B operand of the
@@ -29,6 +31,9 @@
 //  * online softmax in binary32 (exp2 domain) with a lazily updated maximum;
 //    partial results per split are merged by a separate log-sum-exp combine,
 //    except when a row has a single split: its CTA then writes the output;
+//  * the default grid is one CTA per split; the opt-in balanced schedule
+//    (one wave, several spans per CTA) keeps each warp's copy ring running
+//    across spans (see decode_kernel);
 //  * with rotated keys (KVQ_FLAG_ROTATE_KEYS) the prologue turns the query
 //    into H q / D in shared memory;
 //  * paged layout (KVQ_FLAG_PAGED): a stage's 32 positions lie in one page;
@@ -467,7 +472,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
     for (int gr = 0; gr < NGV; ++gr) zacc[hs][gr] = make_float2(0.0f, 0.0f);
 
   {
-    // -------- query fragments (B operand of the score product), once per CTA
+    // -------- query fragments (B operand of the score product), once per span
     // With rotated keys (KVQ_FLAG_ROTATE_KEYS) the query becomes H q / D: the
     // CTA's query rows are transformed in shared memory first (the weight
     // staging buffer is unused until the first tile).
