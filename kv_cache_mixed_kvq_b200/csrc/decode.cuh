@@ -1089,6 +1089,9 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     }
     fence_barrier_init();
   }
+  // the query buffers' barriers and the control words are shared by all
+  // warps: initialised before any warp uses them
+  __syncthreads();
   const int lim = min(a.max_seq_len, a.capacity);
   const bool stream = a.stream_q > 0;
 
