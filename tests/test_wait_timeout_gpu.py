@@ -66,3 +66,34 @@ def test_knob_rejects_out_of_range_limits_and_disarms():
     kvq.kvq_decode_attention(cache, q, lens, 512)
     torch.cuda.synchronize()
     assert kvq.kvq_last_device_error() == 0
+
+
+@pytest.mark.parametrize("drop_stage", [0, 1])
+def test_wait_runs_out_under_the_balanced_schedule(drop_stage, monkeypatch):
+    # one-wave schedule: the first CTA's range crosses a unit boundary (row
+    # 0's units have 3 stages, a CTA takes 4), so when its wait runs out the
+    # next span's query rows and stages may already be in flight; they are
+    # waited for before the CTA ends
+    monkeypatch.setenv("KVQ_DECODE_SCHEDULE", "balanced")
+    B, Hkv, Hq, D, T = 2, 8, 32, 128, 2048
+    cache = _cache(B, Hkv, D, T, seed=7)
+    q = torch.randn(B, Hq, D, generator=torch.Generator().manual_seed(8)).to(
+        torch.bfloat16).cuda()
+    lens = torch.tensor([300, T], dtype=torch.int32, device="cuda")
+    ref = kvq.kvq_decode_attention(cache, q, lens, T, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert kvq.kvq_last_device_error() == 0
+
+    kvq.kvq_debug_inject_wait_timeout(drop_stage, wait_limit_ns=1_000_000)
+    t0 = time.perf_counter()
+    kvq.kvq_decode_attention(cache, q, lens, T, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    flags = kvq.kvq_last_device_error()
+    assert flags & kvq.KVQ_DEVERR_TIMEOUT, f"flags {flags}"
+    assert elapsed < 0.5
+
+    again = kvq.kvq_decode_attention(cache, q, lens, T, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert kvq.kvq_last_device_error() == 0
+    assert torch.equal(again, ref)
