@@ -382,15 +382,16 @@ int32_t kvq_decode_split_tokens(const kvq_cache_desc* cache,
 /*
  * Failure-detection test knob; not for production use.  The summary page has
  * no counterpart: it exists so that a test can make a bounded device wait run
- * out without faulting or hanging the GPU.  With drop_stage >= 0, the next
- * decode-attention launch in this process (only that one) arms stage
- * `drop_stage` of the first warp's copy pipeline in its first CTA without
- * issuing the copies, and every bounded wait of that launch gives up after
- * wait_limit_ns (1000 .. 1e9 ns) instead of one second.  The wait on the
- * dropped stage then runs out: the kernel flags KVQ_DEVERR_TIMEOUT, waits
- * (bounded) for its copies in flight, and returns; that call's output is
- * unspecified, and the cache is untouched.  drop_stage < 0 disarms the knob.
- * Returns KVQ_OK, or KVQ_ERR_INVALID_ARG for a limit out of range.
+ * out without faulting or hanging the GPU.  With drop_stage 0 or 1, the next
+ * decode-attention launch in this process (only that one) makes stage
+ * `drop_stage` of the first warp's copy pipeline in its first CTA expect 16
+ * bytes more than its copies bring, and every bounded wait of that launch
+ * gives up after wait_limit_ns (1000 .. 1e9 ns) instead of one second.  The
+ * wait on that stage then runs out: the kernel flags KVQ_DEVERR_TIMEOUT,
+ * waits (bounded) for its copies in flight, and returns; that call's output
+ * is unspecified, and the cache is untouched.  drop_stage < 0 disarms the
+ * knob.  Returns KVQ_OK, or KVQ_ERR_INVALID_ARG for a stage above 1 or a
+ * limit out of range.
  */
 int kvq_debug_inject_wait_timeout(int32_t drop_stage, int64_t wait_limit_ns);
 

@@ -278,8 +278,9 @@ def kvq_append_decode_attention(cache: KVCache, k_new: torch.Tensor, v_new: torc
 
 
 def kvq_debug_inject_wait_timeout(drop_stage: int, wait_limit_ns: int = 1_000_000) -> None:
-    """Test knob: the next decode launch drops one copy stage so that a bounded
-    wait runs out (see kvq.h); drop_stage < 0 disarms it."""
+    """Test knob: in the next decode launch, stage drop_stage (0 or 1) of the
+    first warp's copy pipeline expects more bytes than its copies bring, so
+    that a bounded wait runs out (see kvq.h); drop_stage < 0 disarms it."""
     _check(library().kvq_debug_inject_wait_timeout(int(drop_stage), int(wait_limit_ns)),
            "kvq_debug_inject_wait_timeout")
 

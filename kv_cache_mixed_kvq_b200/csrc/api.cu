@@ -560,6 +560,7 @@ int kvq_debug_inject_wait_timeout(int32_t drop_stage, int64_t wait_limit_ns) {
     g_fault_stage.store(-1);
     return KVQ_OK;
   }
+  if (drop_stage > 1) return KVQ_ERR_INVALID_ARG;  // only the first two stages are armed
   if (wait_limit_ns < 1000 || wait_limit_ns > 1000000000LL) return KVQ_ERR_INVALID_ARG;
   g_fault_limit_ns.store(wait_limit_ns);
   g_fault_stage.store(drop_stage);

@@ -343,9 +343,6 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
     const uint32_t kbytes = n16 * C::KROW, vbytes = (n16 / 16) * C::VTILE;
     const uint32_t pkbytes = n16 * C::PROWK, pvbytes = n16 * C::PROWV;
     mbar_arrive_expect_tx(&wfull[sl], kbytes + vbytes + pkbytes + pvbytes);
-    if (it == a.fault_stage && warp == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
-        blockIdx.z == 0)
-      return;  // test knob: bytes announced, no copy issued (the wait runs out)
     bulk_copy_g2s(dst, a.k_codes + r * C::KROW, kbytes, &wfull[sl]);
     bulk_copy_g2s(dst + C::SLOT_K, a.v_codes + (r / 16) * C::VTILE, vbytes, &wfull[sl]);
     bulk_copy_g2s(dst + C::SLOT_K + C::SLOT_V,
@@ -356,6 +353,15 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
                   &wfull[sl]);
   };
   int issued = pre;  // stages of the stream from g0 on that are in flight or consumed
+  // Test knob (kvq_debug_inject_wait_timeout): stage `fault_stage` (0 or 1)
+  // of the first warp's stream in the first CTA expects 16 bytes more than
+  // its copies bring, so that the wait on it runs out.  Checked only where
+  // the first stages are requested, never in the main loop.
+  auto knob = [&](int stream_stage, int sl) {
+    if (stream_stage == a.fault_stage && warp == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
+        blockIdx.z == 0)
+      mbar_expect_tx(&wfull[sl], 16);
+  };
   // the next span's query rows
   const bool q_bulk = !a.rotate_q;
   uint8_t* qbuf = smem + C::QBUF_OFF;
@@ -406,12 +412,15 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
           first_pending = it;
           break;
         }
+        knob(g0 + it, (g0 + it) % C::kSlots);
         issue(cur, it, (g0 + it) % C::kSlots, a.block_table != nullptr ? page_of(cur, it) : 0);
       }
     } else {
-      for (; issued < min(C::kSlots, my_iters); ++issued)
+      for (; issued < min(C::kSlots, my_iters); ++issued) {
+        knob(g0 + issued, (g0 + issued) % C::kSlots);
         issue(cur, issued, (g0 + issued) % C::kSlots,
               a.block_table != nullptr ? page_of(cur, issued) : 0);
+      }
     }
   }
   if constexpr (FUSED) {
@@ -438,8 +447,10 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
       }
     }
     if (lane == 0)
-      for (int it = first_pending; it < min(C::kSlots, my_iters); ++it)
+      for (int it = first_pending; it < min(C::kSlots, my_iters); ++it) {
+        knob(g0 + it, (g0 + it) % C::kSlots);
         issue(cur, it, (g0 + it) % C::kSlots, a.block_table != nullptr ? page_of(cur, it) : 0);
+      }
     issued = min(C::kSlots, my_iters);
   }
   __syncwarp();

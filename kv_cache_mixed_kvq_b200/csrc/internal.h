@@ -84,8 +84,8 @@ struct DecodeArgs {
   const void* v_new;
   int in_dtype, n_new;
   // Failure-detection test knob (kvq_debug_inject_wait_timeout): when
-  // fault_stage >= 0, the first CTA's first warp arms that stage of its copy
-  // pipeline without issuing its copies, so that the wait on it runs out;
+  // fault_stage is 0 or 1, that stage of the first CTA's first warp expects
+  // 16 bytes more than its copies bring, so that the wait on it runs out;
   // every bounded wait of the launch gives up after wait_limit_ns.
   int fault_stage;
   unsigned long long wait_limit_ns;

@@ -157,5 +157,6 @@ def test_fused_append_rejects_before_launch():
 def test_wait_timeout_knob_is_validated_on_the_host():
     lib = kvq.library()
     assert lib.kvq_debug_inject_wait_timeout(0, 10) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_debug_inject_wait_timeout(2, 1_000_000) == kvq.KVQ_ERR_INVALID_ARG
     assert lib.kvq_debug_inject_wait_timeout(0, 2_000_000_000) == kvq.KVQ_ERR_INVALID_ARG
     assert lib.kvq_debug_inject_wait_timeout(-1, 0) == kvq.KVQ_OK

@@ -1,9 +1,9 @@
 """Failure detection on the GPU without a fault: a bounded wait that runs out.
 
 Every wait of the decode kernel's copy pipeline is bounded.  The test knob
-kvq_debug_inject_wait_timeout() makes the next decode launch announce the
-bytes of one pipeline stage on its mbarrier without issuing the copies, and
-shortens the wait limit to one millisecond.  The wait on that stage then runs
+kvq_debug_inject_wait_timeout() makes one of the first two pipeline stages of
+the next decode launch expect more bytes on its mbarrier than its copies
+bring, and shortens the wait limit to one millisecond.  The wait on that stage then runs
 out: the kernel must flag KVQ_DEVERR_TIMEOUT, drain its other copies and
 return (no hang, no fault), and the context must stay usable: the next
 normal call on the same cache reproduces a fresh call bit for bit.
@@ -57,7 +57,7 @@ def test_wait_runs_out_flags_timeout_and_recovers(drop_stage):
 def test_knob_rejects_out_of_range_limits_and_disarms():
     with pytest.raises(kvq.KvqError):
         kvq.kvq_debug_inject_wait_timeout(0, wait_limit_ns=10)
-    kvq.kvq_debug_inject_wait_timeout(2, wait_limit_ns=1_000_000)
+    kvq.kvq_debug_inject_wait_timeout(1, wait_limit_ns=1_000_000)
     kvq.kvq_debug_inject_wait_timeout(-1)  # disarmed: the next call is normal
     cache = _cache(1, 8, 128, 512, seed=5)
     q = torch.randn(1, 32, 128, generator=torch.Generator().manual_seed(6)).to(
