@@ -176,8 +176,10 @@ bool select_decode_kernel(const kvq_cache_desc* c, int heads_per_cta, int q_dtyp
   const int gk = c->head_dim / c->group, gv = c->head_dim / group_v_of(c);
   if (use_tc_kernel(c, fused))
     return kvq::get_decode_tc_kernel(c->bits_k, c->bits_v, gk, gv, heads_per_cta, k);
+  // variant bit 2 selects the paged layout's instances
+  const int paged = (c->flags & KVQ_FLAG_PAGED) != 0 ? 4 : 0;
   return kvq::get_decode_kernel(c->head_dim, c->bits_k, c->bits_v, gk, gv,
-                                variant_of(heads_per_cta, q_dtype), k);
+                                variant_of(heads_per_cta, q_dtype) | paged, k);
 }
 
 // Opt a kernel in to more than 48 KB of dynamic shared memory, once per

@@ -235,6 +235,18 @@ __device__ __forceinline__ void lds_param_pair(const uint32_t* p, uint32_t (&w0)
   }
 }
 
+// Paged layout or slot layout: fixed at compile time in the plain instances;
+// tested at run time in the fused ones, whose append prologue keeps its
+// registers and schedule best that way (measured: the Qwen-shaped fused step
+// took 77 us with the layout fixed at compile time against 65 us).
+template <bool FUSED, bool PAGED>
+__device__ __forceinline__ bool paged_layout(const DecodeArgs& a) {
+  if constexpr (FUSED)
+    return a.block_table != nullptr;
+  else
+    return PAGED;
+}
+
 // One span of a CTA's work: positions [t0, t1) of (batch row b, kv head hk,
 // head group hg); app_pos: first position the fused append writes (-1:
 // none); the result is the rows' final output (direct) or the partial result
@@ -264,7 +276,9 @@ __device__ __forceinline__ void issue_q_rows(const DecodeArgs& a, const Span& s,
 
 // FUSED: the instance used by the fused append + decode call (the append
 // prologue is compiled only there, so the plain decode keeps its registers
-// and schedule).
+// and schedule).  PAGED: the instance for the paged layout (block-table
+// lookups); the slot layout's instances are compiled without them (their
+// per-stage checks cost 3 % of the steady-state decode).
 // One span cur: the copy pipeline, the online softmax and the four warps'
 // merge.  Each warp's copies form one stream over the CTA's spans: stage g of
 // the stream lands in slot g mod kSlots with phase parity (g / kSlots) mod 2.
@@ -281,7 +295,7 @@ __device__ __forceinline__ void issue_q_rows(const DecodeArgs& a, const Span& s,
 // transform their own copy of the rows instead).
 // Returns true when a wait ran out (the CTA then stops; the rows are
 // flagged).
-template <class C, bool FUSED, class PeekFn, class NextFn>
+template <class C, bool FUSED, bool PAGED, class PeekFn, class NextFn>
 __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, const Span& cur,
                                             PeekFn&& peek, NextFn&& next, Span& nxt,
                                             bool& has_next, int ws_stride, int& g0, int& pre) {
@@ -302,6 +316,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
   const int nh = min(a.heads_per_cta, a.gq - hg * a.heads_per_cta);
   const int n_tok = t1 - t0;
   const size_t slot = static_cast<size_t>(b) * a.kv_heads + hk;
+  const bool paged = paged_layout<FUSED, PAGED>(a);
 
   // ---- this warp's copy pipeline: positions [it*kStageTokens + 16*TPW*warp, +16*TPW)
   // of a span for it = 0 .. iters-1, kSlots copies in flight.
@@ -329,7 +344,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
     const int tb = s.t0 + base;
     uint8_t* dst = wring + sl * C::SLOT_BYTES;
     size_t r = (static_cast<size_t>(s.b) * a.kv_heads + s.hk) * a.capacity + tb;
-    if (a.block_table != nullptr) {
+    if (paged) {
       if (page < 0 || page >= a.num_pages) {
         // no page: nothing is read (the row's output is unspecified); the
         // stage completes at once so that the pipeline keeps going
@@ -381,7 +396,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
   // t0, t1; b < 0: none), kept in shared memory rather than registers (read
   // through a volatile pointer, so that the reads stay where they are used)
   volatile int* wnext = ctl + 4 + 4 * warp;
-  if (!FUSED && a.block_table == nullptr && lane == 0) {
+  if (!FUSED && !paged && lane == 0) {
     Span s;
     const bool any = peek(s);
     wnext[0] = any ? s.b : -1;
@@ -413,13 +428,13 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
           break;
         }
         knob(g0 + it, (g0 + it) % C::kSlots);
-        issue(cur, it, (g0 + it) % C::kSlots, a.block_table != nullptr ? page_of(cur, it) : 0);
+        issue(cur, it, (g0 + it) % C::kSlots, paged ? page_of(cur, it) : 0);
       }
     } else {
       for (; issued < min(C::kSlots, my_iters); ++issued) {
         knob(g0 + issued, (g0 + issued) % C::kSlots);
         issue(cur, issued, (g0 + issued) % C::kSlots,
-              a.block_table != nullptr ? page_of(cur, issued) : 0);
+              paged ? page_of(cur, issued) : 0);
       }
     }
   }
@@ -432,7 +447,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
       const int p0 = max(app_pos, t0), p1 = t1;
       if (p0 < p1) {
         auto row_of_pos = [&](int p) -> long long {
-          if (a.block_table == nullptr) return static_cast<long long>(slot) * a.capacity + p;
+          if (!paged) return static_cast<long long>(slot) * a.capacity + p;
           const int page =
               a.block_table[static_cast<size_t>(b) * a.pages_per_seq + (p >> a.page_shift)];
           if (page < 0 || page >= a.num_pages) return -1;
@@ -449,7 +464,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
     if (lane == 0)
       for (int it = first_pending; it < min(C::kSlots, my_iters); ++it) {
         knob(g0 + it, (g0 + it) % C::kSlots);
-        issue(cur, it, (g0 + it) % C::kSlots, a.block_table != nullptr ? page_of(cur, it) : 0);
+        issue(cur, it, (g0 + it) % C::kSlots, paged ? page_of(cur, it) : 0);
       }
     issued = min(C::kSlots, my_iters);
   }
@@ -918,7 +933,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
       // arithmetic so that the block-table read overlaps it
       const bool refill = it + C::kSlots < my_iters;
       int next_page = 0;
-      if (a.block_table != nullptr && lane == 0 && refill) next_page = page_of(cur, it + C::kSlots);
+      if (paged && lane == 0 && refill) next_page = page_of(cur, it + C::kSlots);
       if (!mbar_wait_bounded(&wfull[sl], phase, err, a.wait_limit_ns)) break;
       const uint8_t* st = wring + sl * C::SLOT_BYTES;
       const int base = it * C::kStageTokens + my_first;  // first position of this slot
@@ -943,7 +958,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
           fence_proxy_async_shared();
           issue(cur, it + C::kSlots, sl, next_page);
           ++issued;
-        } else if (!FUSED && a.block_table == nullptr && it + C::kSlots == issued &&
+        } else if (!FUSED && !paged && it + C::kSlots == issued &&
                    wnext[0] >= 0) {
           Span s;
           s.b = wnext[0];
@@ -974,7 +989,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
     const int n = min(C::kSlots, iters_of(nxt));
     for (; issued < my_iters + n; ++issued)
       issue(nxt, issued - my_iters, (g0 + issued) % C::kSlots,
-            a.block_table != nullptr ? page_of(nxt, issued - my_iters) : 0);
+            paged ? page_of(nxt, issued - my_iters) : 0);
   }
 
   // ------------------------------------------------------------ epilogue
@@ -1079,7 +1094,7 @@ __device__ __forceinline__ bool decode_span(const DecodeArgs& a, uint8_t* smem, 
 // directly; the others leave one partial result per covering CTA (index:
 // the CTA's rank among them) for the combine kernel.  The balanced schedule
 // takes at most kStreamRows rows.
-template <class C, bool FUSED>
+template <class C, bool FUSED, bool PAGED>
 __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     decode_kernel(const DecodeArgs a) {
   constexpr int D = C::D, T = C::kStageTokens;
@@ -1234,7 +1249,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     if (!first) __syncthreads();
     Span nxt = cur;
     bool has_next = false;
-    if (decode_span<C, FUSED>(a, smem, cur, peek, next, nxt, has_next, a.num_splits, g0, pre) ||
+    if (decode_span<C, FUSED, PAGED>(a, smem, cur, peek, next, nxt, has_next, a.num_splits, g0,
+                                     pre) ||
         !has_next)
       break;
     cur = nxt;
@@ -1249,20 +1265,21 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
   }
 }
 
-template <class C, bool FUSED>
+template <class C, bool FUSED, bool PAGED>
 cudaError_t launch_decode(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
-  return launch_pdl(decode_kernel<C, FUSED>, grid, dim3(C::kThreads), C::SMEM_BYTES, stream, a);
+  return launch_pdl(decode_kernel<C, FUSED, PAGED>, grid, dim3(C::kThreads), C::SMEM_BYTES,
+                    stream, a);
 }
 
-template <class C>
+template <class C, bool PAGED>
 DecodeKernel make_decode_kernel() {
   DecodeKernel k;
-  k.fn = reinterpret_cast<const void*>(&decode_kernel<C, false>);
-  k.fn_fused = reinterpret_cast<const void*>(&decode_kernel<C, true>);
+  k.fn = reinterpret_cast<const void*>(&decode_kernel<C, false, PAGED>);
+  k.fn_fused = reinterpret_cast<const void*>(&decode_kernel<C, true, PAGED>);
   k.threads = C::kThreads;
   k.smem_bytes = C::SMEM_BYTES;
-  k.launch = &launch_decode<C, false>;
-  k.launch_fused = &launch_decode<C, true>;
+  k.launch = &launch_decode<C, false, PAGED>;
+  k.launch_fused = &launch_decode<C, true, PAGED>;
   k.tile = 64;
   k.max_per_sm = 0;
   k.stage_tokens = C::kStageTokens;
@@ -1275,15 +1292,17 @@ DecodeKernel make_decode_kernel() {
 // query variants: up to 4 heads per CTA (any query type: one head per lane,
 // high/low columns), 5..8 heads with 16-bit queries (two heads per lane),
 // 5..8 heads with binary32 queries (high/low columns, two n-tiles).
-template <int BK, int BV>
+// PAGED: the paged layout's instances (compiled in their own translation
+// units, so that the two families build in parallel).
+template <int BK, int BV, bool PAGED>
 bool get_decode_kernel_bits(int head_dim, int groups_k, int groups_v, int variant,
                             DecodeKernel* out) {
 #define KVQ_VARIANTS(D, NGK, NGV)                                                          \
   switch (variant) {                                                                       \
     case 0:                                                                                \
-    case 1: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NGK, NGV, 2, 1, 1>>(); return true; \
-    case 2: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NGK, NGV, 1, 1, 2>>(); return true; \
-    case 3: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NGK, NGV, 2, 2, 2>>(); return true; \
+    case 1: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NGK, NGV, 2, 1, 1>, PAGED>(); return true; \
+    case 2: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NGK, NGV, 1, 1, 2>, PAGED>(); return true; \
+    case 3: *out = make_decode_kernel<DecodeCfg<D, BK, BV, NGK, NGV, 2, 2, 2>, PAGED>(); return true; \
     default: return false;                                                                 \
   }
 #define KVQ_GROUPS(D, NGK, NGV) \

@@ -2,8 +2,13 @@
 #include "decode.cuh"
 
 namespace kvq {
+bool get_decode_kernel_k2v8_paged(int head_dim, int groups_k, int groups_v, int variant,
+                                  DecodeKernel* out);
+
+// variant bit 2: the paged layout's instances (decode_k2v8_paged.cu)
 bool get_decode_kernel_k2v8(int head_dim, int groups_k, int groups_v, int variant,
                             DecodeKernel* out) {
-  return get_decode_kernel_bits<2, 8>(head_dim, groups_k, groups_v, variant, out);
+  if (variant & 4) return get_decode_kernel_k2v8_paged(head_dim, groups_k, groups_v, variant & 3, out);
+  return get_decode_kernel_bits<2, 8, false>(head_dim, groups_k, groups_v, variant, out);
 }
 }  // namespace kvq

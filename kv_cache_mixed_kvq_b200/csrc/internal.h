@@ -114,7 +114,8 @@ struct DecodeKernel {
   cudaError_t (*launch_fused)(const DecodeArgs&, dim3 grid, cudaStream_t stream);
 };
 
-// Returns false if (D, bits, key groups, value groups, variant) has no instance.
+// Returns false if (D, bits, key groups, value groups, variant) has no instance
+// (variant bits 0-1: query-head variant; bit 2: the paged layout's instances).
 bool get_decode_kernel(int head_dim, int bits_k, int bits_v, int groups_k, int groups_v,
                        int variant, DecodeKernel* out);
 
