@@ -560,56 +560,94 @@ def per_kernel_times(arm, rotate, reps):
 def run_e2e(arm, args, step_bytes, world, device):
     """Same step through the public API with pinned host buffers: H2D of the
     step's inputs (query, lengths and any new K/V rows), the step's calls,
-    D2H of the output, every step.  The cache is the step's resident state."""
+    D2H of the output, every step.  The cache is the step's resident state.
+
+    The steps are pipelined the way a serving loop would run them: the
+    inputs and the output of each step have two device buffers, copies go on
+    their own streams, so that step i+1's inputs come in and step i-1's
+    output goes out while step i computes; events order every buffer's
+    reuse.  The timed region starts before the first copy in and ends after
+    the last copy out."""
     s0 = arm.sets[0]
     hk = s0["k"].cpu().pin_memory()
     hv = s0["v"].cpu().pin_memory()
     hq = s0["q"].cpu().pin_memory()
     hlens = arm.lens.cpu().pin_memory()
-    hout = torch.empty_like(s0["out"], device="cpu").pin_memory()
-    k_dev, v_dev, q_dev = torch.empty_like(s0["k"]), torch.empty_like(s0["v"]), torch.empty_like(s0["q"])
-    lens_dev = torch.empty_like(arm.lens)
+    hout = [torch.empty_like(s0["out"], device="cpu").pin_memory() for _ in range(2)]
+    bufs = [{"k": torch.empty_like(s0["k"]), "v": torch.empty_like(s0["v"]),
+             "q": torch.empty_like(s0["q"]), "lens": torch.empty_like(arm.lens),
+             "out": torch.empty_like(s0["out"])} for _ in range(2)]
     cache = s0["cache"]
-    stream = torch.cuda.current_stream()
+    comp = torch.cuda.current_stream()
+    cin, cout = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()  # noqa: E731  (ordering only)
+    in_ready, comp_done, out_done = ([ev(), ev()] for _ in range(3))
+    used = [False, False]
 
-    def one():
-        if arm.n_new:
-            k_dev.copy_(hk, non_blocking=True)
-            v_dev.copy_(hv, non_blocking=True)
-        q_dev.copy_(hq, non_blocking=True)
-        lens_dev.copy_(hlens, non_blocking=True)
+    def one(i):
+        sl, d = i % 2, bufs[i % 2]
+        with torch.cuda.stream(cin):
+            if used[sl]:
+                cin.wait_event(comp_done[sl])  # step i-2 has read these inputs
+            if arm.n_new:
+                d["k"].copy_(hk, non_blocking=True)
+                d["v"].copy_(hv, non_blocking=True)
+            d["q"].copy_(hq, non_blocking=True)
+            d["lens"].copy_(hlens, non_blocking=True)
+            in_ready[sl].record(cin)
+        comp.wait_event(in_ready[sl])
+        if used[sl]:
+            comp.wait_event(out_done[sl])  # step i-2's output has left
         if arm.fused:
-            arm.kvq.kvq_append_decode_attention(cache, k_dev, v_dev, q_dev, lens_dev,
-                                                arm.max_len, out=s0["out"], workspace=arm.ws)
+            arm.kvq.kvq_append_decode_attention(cache, d["k"], d["v"], d["q"], d["lens"],
+                                                arm.max_len, out=d["out"], workspace=arm.ws,
+                                                stream=comp)
         else:
             if arm.n_new:
-                arm.kvq.kvq_quantize_append(cache, k_dev, v_dev, arm.pos_t)
-            arm.kvq.kvq_decode_attention(cache, q_dev, lens_dev, arm.max_len, out=s0["out"],
-                                         workspace=arm.ws)
-        hout.copy_(s0["out"], non_blocking=True)
+                arm.kvq.kvq_quantize_append(cache, d["k"], d["v"], arm.pos_t, stream=comp)
+            arm.kvq.kvq_decode_attention(cache, d["q"], d["lens"], arm.max_len, out=d["out"],
+                                         workspace=arm.ws, stream=comp)
+        comp_done[sl].record(comp)
+        with torch.cuda.stream(cout):
+            cout.wait_event(comp_done[sl])
+            hout[sl].copy_(d["out"], non_blocking=True)
+            out_done[sl].record(cout)
+        used[sl] = True
 
-    for _ in range(args.warmup):
-        one()
+    def run(n, start=None):
+        used[0] = used[1] = False
+        if start is not None:
+            start.record(comp)
+            cin.wait_stream(comp)
+        for i in range(n):
+            one(i)
+        comp.wait_stream(cout)
+        comp.wait_stream(cin)
+
+    run(args.warmup)
     torch.cuda.synchronize()
     steps = max(3, min(args.steps, 20))
     if world > 1:
         torch.distributed.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    run(steps, start=a)
+    b.record(comp)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b) / steps, world, device)
+    # the last step's output, as copied out, is the step's result
+    if not torch.equal(hout[(steps - 1) % 2], bufs[(steps - 1) % 2]["out"].cpu()):
+        raise RuntimeError("e2e: the output copied out differs from the device output")
     h2d = hq.numel() * hq.element_size() + hlens.numel() * hlens.element_size()
     if arm.n_new:
         h2d += hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
     return {"value": round(world * step_bytes / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 4), "steps": steps,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout[0].numel() * hout[0].element_size(),
             "what": "the same step through the public API: pinned host query and lengths "
                     "(and new K/V rows when the step appends) copied in, the output copied "
-                    "out, every step; the cache stays resident on the device"}
+                    "out, every step, double-buffered on copy streams so that the copies "
+                    "overlap the neighbouring steps' kernels; the cache stays resident on "
+                    "the device"}
 
 
 # ---------------------------------------------------------- oracle (CPU)
