@@ -503,8 +503,12 @@ int decode_impl(const kvq_cache_desc* cache, const void* k_new, const void* v_ne
     a.out_dtype = out_dtype;
     st = error_word(&a.err);
     if (st != KVQ_OK) return st;
-    const dim3 grid = balanced ? dim3(p.stream_grid, 1, 1)
-                             : dim3(p.num_splits, cache->kv_heads * p.head_groups, cache->batch);
+    // (the fused instance takes the split grid as (units, rows, splits),
+    // each row's last split first: see the decode kernel)
+    const int units = cache->kv_heads * p.head_groups;
+    const dim3 grid = balanced         ? dim3(p.stream_grid, 1, 1)
+                      : k_new != nullptr ? dim3(units, cache->batch, p.num_splits)
+                                         : dim3(p.num_splits, units, cache->batch);
     if ((k_new != nullptr ? k.launch_fused : k.launch)(a, grid, s) != cudaSuccess)
       return KVQ_ERR_CUDA;
     if (a.direct) return KVQ_OK;

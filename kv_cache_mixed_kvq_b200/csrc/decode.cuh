@@ -1184,26 +1184,36 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     stream_span(p, rb, cur, adv);
     first_q();
   } else {
-    const int split = blockIdx.x;
-    cur.hk = blockIdx.y / a.head_groups;
-    cur.hg = blockIdx.y % a.head_groups;
-    cur.b = blockIdx.z;
+    // Grid (splits, kv heads x head groups, batch rows).  The fused instance
+    // is launched as (kv heads x head groups, batch rows, k) instead, split
+    // = the row's last split - k: the splits holding the new positions
+    // (longer than the others by their append) are the first ones the block
+    // scheduler starts, so that none of them ends a later wave.  Same
+    // splits, same results; only the launch order differs.
+    const int unit = FUSED ? blockIdx.x : blockIdx.y;
+    const int k = FUSED ? blockIdx.z : blockIdx.x;  // k == 0: one CTA per row flags
+    cur.hk = unit / a.head_groups;
+    cur.hg = unit % a.head_groups;
+    cur.b = FUSED ? blockIdx.y : blockIdx.z;
     int len = a.seq_lens[cur.b];
     // fused append: positions [len - n_new, len) are written first; a row
     // whose length is out of range appends nothing
     cur.app_pos = -1;
     if (FUSED && a.k_new != nullptr && len <= lim) {
       if (len < a.n_new) {
-        if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0)
-          flag_error(a.err, KVQ_DEVERR_BAD_POS);
+        if (k == 0 && unit == 0 && threadIdx.x == 0) flag_error(a.err, KVQ_DEVERR_BAD_POS);
       } else {
         cur.app_pos = len - a.n_new;
       }
     }
     if (len < 0 || len > lim) {
-      if (split == 0 && blockIdx.y == 0 && threadIdx.x == 0)
-        flag_error(a.err, KVQ_DEVERR_SEQ_LEN);
+      if (k == 0 && unit == 0 && threadIdx.x == 0) flag_error(a.err, KVQ_DEVERR_SEQ_LEN);
       len = max(0, min(len, lim));
+    }
+    int split = k;
+    if constexpr (FUSED) {
+      const int ns = (len + a.split_tokens - 1) / a.split_tokens;
+      if (k < ns) split = ns - 1 - k;  // (k >= ns: past the row, empty as on the plain grid)
     }
     cur.t0 = split * a.split_tokens;
     if (cur.t0 >= len) {

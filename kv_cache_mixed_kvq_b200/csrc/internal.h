@@ -69,7 +69,7 @@ struct DecodeArgs {
   int heads_per_cta;  // <= 8
   int head_groups;    // ceil(gq / heads_per_cta)
   int split_tokens;   // multiple of 64
-  int num_splits;     // grid.x; balanced schedule: partial slots per row
+  int num_splits;     // splits per row (grid.x; grid.z of the fused instance); balanced schedule: partial slots per row
   // Balanced (stream-K) schedule when > 0: grid.x CTAs share the rows' stages
   // evenly, at least stream_q stages each (plain decode only).
   int stream_q;
