@@ -19,13 +19,16 @@ algorithmic bytes, GB/s and fraction of the measured HBM copy bandwidth.
 
 Timing: inputs and caches rotate over enough sets that the data touched
 between two uses of a set exceeds twice the L2 (the device's own L2 size);
-each step is replayed from a CUDA graph; the timed region is bracketed by a
+the steps are replayed from a CUDA graph holding one step of every set in
+order (consecutive steps chain through programmatic dependent launch, as
+consecutive decode calls on a stream do; --step-graphs single replays one
+graph per step instead); the timed region is bracketed by a
 barrier and a device synchronize, timed with CUDA events on the launch
 stream, max over ranks.  Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME] [--bits K,V] [--group-v G] [--rotate-keys]
-                  [--page-size P] [--fused] [--no-configs]
+                  [--page-size P] [--fused] [--no-configs] [--step-graphs chain|single]
 """
 from __future__ import annotations
 
@@ -397,15 +400,28 @@ def run_ours(args, rank, world, device):
     if flags:
         raise RuntimeError(f"device error flags {flags} during warm-up")
 
-    # one CUDA graph per rotation set
+    # one CUDA graph per rotation set, and (--step-graphs chain) one graph of
+    # all the sets' steps in order: inside it consecutive steps chain through
+    # programmatic dependent launch, as consecutive decode calls on a stream
+    # do (each step's kernels still wait for the previous step's to finish
+    # before touching memory)
     graphs = []
     for r in range(rotate):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             arm.step(r)
         graphs.append(g)
+    chain = None
+    if args.step_graphs == "chain" and rotate > 1:
+        chain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(chain):
+            for r in range(rotate):
+                arm.step(r)
+        graphs.append(chain)  # (released with the others)
     for i in range(args.warmup):
         graphs[i % rotate].replay()
+    if chain is not None:
+        chain.replay()
     torch.cuda.synchronize()
 
     # ---------------- timed region: exactly K steps
@@ -416,7 +432,10 @@ def run_ours(args, rank, world, device):
     t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(physical_index()) as clocks:
         t0.record(stream)
-        for i in range(args.steps):
+        n_chain, rest = divmod(args.steps, rotate) if chain is not None else (0, args.steps)
+        for _ in range(n_chain):
+            chain.replay()  # `rotate` steps
+        for i in range(rest):
             graphs[i % rotate].replay()
         t1.record(stream)
         torch.cuda.synchronize()
@@ -454,7 +473,9 @@ def run_ours(args, rank, world, device):
         "split_tokens": arm.split_tokens,
         "l2": f"{rotate} rotating input/cache sets of {step_bytes / 1e6:.1f} MB (each "
               f"step's data last touched {rotate - 1} steps earlier; L2 "
-              f"{l2_bytes(device) / 2**20:.0f} MiB), graph replay",
+              f"{l2_bytes(device) / 2**20:.0f} MiB), graph replay"
+              + (f" ({rotate} consecutive steps per graph)" if chain is not None
+                 else " (one step per graph)"),
         "parallelism": f"replicas{world}" if world > 1 else "single",
     }
     if w.ragged:
@@ -848,6 +869,9 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--step-graphs", choices=["chain", "single"], default="chain",
+                    help="timed steps replayed from one graph per rotating set (single) or "
+                         "from one graph holding every set's step in order (chain)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
