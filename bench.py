@@ -152,14 +152,20 @@ def max_over_ranks(x: float, world: int, device) -> float:
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
+    """nvidia-smi samples every 100 ms while the context is open.  With
+    window(t0, t1) (host wall-clock seconds), summary() keeps only the
+    samples taken inside [t0, t1]: the ones under load."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "timestamp")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, lead: float = 0.3):
         self.idx = device_index
+        self.lead = lead
         self.proc = None
         self.file = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
@@ -168,10 +174,22 @@ class ClockSampler:
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.file, stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
+            time.sleep(self.lead)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
+
+    def window(self, t0: float, t1: float):
+        self.t0, self.t1 = t0, t1
+
+    def _in_window(self, row) -> bool:
+        if self.t0 is None:
+            return True
+        try:
+            ts = datetime.datetime.strptime(row[9], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except (IndexError, ValueError):
+            return False
+        return self.t0 <= ts <= self.t1
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -189,14 +207,19 @@ class ClockSampler:
         self.file.seek(0)
         rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
         rows = [[x.strip() for x in r] for r in rows if len(r) >= 9]
+        rows = [r for r in rows if self._in_window(r)]
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None,
+               "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        if self.t0 is not None:
+            out["window"] = (f"{self.t1 - self.t0:.2f} s: the same steps untimed for 1 s, then "
+                             f"the timed region")
+        return out
 
 
 # -------------------------------------------------------------- our arm
@@ -430,7 +453,18 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(physical_index()) as clocks:
+    with ClockSampler(physical_index(), lead=0.0) as clocks:
+        # the same steps, untimed, for a second before the timed region, so
+        # that the clock samples (every 100 ms) are taken under this load:
+        # the timed region itself is shorter than one sampling interval
+        load_start = time.time()
+        while time.time() < load_start + 1.0:
+            for g in graphs[:rotate]:
+                g.replay()
+            torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
         t0.record(stream)
         n_chain, rest = divmod(args.steps, rotate) if chain is not None else (0, args.steps)
         for _ in range(n_chain):
@@ -439,6 +473,7 @@ def run_ours(args, rank, world, device):
             graphs[i % rotate].replay()
         t1.record(stream)
         torch.cuda.synchronize()
+        clocks.window(load_start, time.time())
     if world > 1:
         torch.distributed.barrier()
     ms = max_over_ranks(t0.elapsed_time(t1), world, device)

@@ -2,6 +2,7 @@
 behind every GB/s figure, the max-over-ranks reduction of the timed region
 (world size 2 over gloo), and the reference arm's launch under torchrun
 (rank 0 alone prints one JSON line, the other rank exits 0)."""
+import datetime
 import json
 import os
 import socket
@@ -137,3 +138,25 @@ def test_config_sweep_covers_every_workload_and_bit_pair():
     appending = {n for n, w in bench.workloads.WORKLOADS.items() if w.append > 0}
     assert fused == appending
     assert bench.DEFAULT_WORKLOAD == "ragged" and bench.KERNEL_REPS >= 50
+
+
+def test_clock_summary_keeps_only_samples_inside_the_window(tmp_path):
+    # nvidia-smi rows (csv, no header, no units): index, sm clock, max clock,
+    # power, active reasons, four reason flags, timestamp
+    def row(t, mhz, cap="Not Active"):
+        ts = datetime.datetime.fromtimestamp(t).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"0, {mhz}, 1965, 600.0, 0x0, Not Active, Not Active, Not Active, {cap}, {ts}"
+
+    t = 1_800_000_000.0
+    f = open(tmp_path / "clocks.csv", "w+")
+    f.write("\n".join([row(t - 0.5, 900), row(t + 0.1, 1965), row(t + 0.2, 1950, "Active"),
+                       row(t + 2.0, 1000)]) + "\n")
+    s = bench.ClockSampler(0, lead=0.0)
+    s.proc, s.file = object(), f
+    s.window(t, t + 1.0)
+    out = s.summary()
+    assert out["samples"] == 2
+    assert out["sm_mhz"] == (1965 + 1950) / 2
+    assert out["reasons"] == ["sw_power_cap"]
+    s.t0 = None  # no window: every sample
+    assert s.summary()["samples"] == 4
