@@ -1188,8 +1188,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     // is launched as (kv heads x head groups, batch rows, k) instead, split
     // = the row's last split - k: the splits holding the new positions
     // (longer than the others by their append) are the first ones the block
-    // scheduler starts, so that none of them ends a later wave.  Same
-    // splits, same results; only the launch order differs.
+    // scheduler starts and places.  Same splits, same results; only the
+    // launch order differs.
     const int unit = FUSED ? blockIdx.x : blockIdx.y;
     const int k = FUSED ? blockIdx.z : blockIdx.x;  // k == 0: one CTA per row flags
     cur.hk = unit / a.head_groups;
