@@ -370,6 +370,16 @@ def kernel_rooflines(arm, w, kern, nbytes, reps, rotate_keys=False):
     return roof
 
 
+def timed_replays(steps, rotate, chained):
+    """The graph replays of the timed region, in order: None for the graph
+    of `rotate` consecutive steps (sets 0 .. rotate-1), r for set r's
+    single-step graph.  Exactly `steps` steps, sets taken in turn."""
+    if not chained:
+        return [i % rotate for i in range(steps)]
+    n_chain, rest = divmod(steps, rotate)
+    return [None] * n_chain + list(range(rest))
+
+
 def in_region_roofline(arm, entry, ms_step):
     """When the timed step is the decode-attention call alone (no separate
     quantize launch), its average duration over the timed region is the
@@ -479,11 +489,8 @@ def run_ours(args, rank, world, device):
             torch.distributed.barrier()
         torch.cuda.synchronize()
         t0.record(stream)
-        n_chain, rest = divmod(args.steps, rotate) if chain is not None else (0, args.steps)
-        for _ in range(n_chain):
-            chain.replay()  # `rotate` steps
-        for i in range(rest):
-            graphs[i % rotate].replay()
+        for g in timed_replays(args.steps, rotate, chain is not None):
+            (chain if g is None else graphs[g]).replay()
         t1.record(stream)
         torch.cuda.synchronize()
         clocks.window(load_start, time.time())

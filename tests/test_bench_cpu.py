@@ -160,3 +160,14 @@ def test_clock_summary_keeps_only_samples_inside_the_window(tmp_path):
     assert out["reasons"] == ["sw_power_cap"]
     s.t0 = None  # no window: every sample
     assert s.summary()["samples"] == 4
+
+
+def test_timed_replays_run_exactly_k_steps_in_set_order():
+    for rotate in (1, 2, 3, 5):
+        for steps in (1, 2, 3, 7, 50):
+            for chained in (False, True):
+                order = []
+                for g in bench.timed_replays(steps, rotate, chained and rotate > 1):
+                    order.extend(range(rotate) if g is None else [g])
+                assert len(order) == steps
+                assert order == [i % rotate for i in range(steps)]
