@@ -232,9 +232,10 @@ def kvq_decode_attention(cache: KVCache, q: torch.Tensor, seq_lens: torch.Tensor
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     d = cache.desc()
     lib = library()
-    need = int(lib.kvq_decode_workspace_bytes(ctypes.byref(d), q.shape[1], max_seq_len))
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:  # (a given workspace is checked by the library itself)
+        need = int(lib.kvq_decode_workspace_bytes(ctypes.byref(d), q.shape[1], max_seq_len))
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev_ptr(workspace, "workspace") if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = lib.kvq_decode_attention(ctypes.byref(d), _dev_ptr(q, "q"), _DTYPE[q.dtype], q.shape[1],
@@ -263,9 +264,10 @@ def kvq_append_decode_attention(cache: KVCache, k_new: torch.Tensor, v_new: torc
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     d = cache.desc()
     lib = library()
-    need = int(lib.kvq_decode_workspace_bytes(ctypes.byref(d), q.shape[1], max_seq_len))
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:  # (a given workspace is checked by the library itself)
+        need = int(lib.kvq_decode_workspace_bytes(ctypes.byref(d), q.shape[1], max_seq_len))
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev_ptr(workspace, "workspace") if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = lib.kvq_append_decode_attention(
